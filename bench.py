@@ -1,0 +1,315 @@
+"""Benchmark of the W4A4 NVFP4 hot path on B200.
+
+One step = one pass of the per-call hot path over one batch of synthetic
+prefill activations:  fp4_quantize_act (amax pass + fused block quantizer,
+DYNAMIC global scale, MMA scale order)  ->  fp4_gemm (tcgen05 block-scaled
+GEMM, alpha epilogue, bf16 out).  Weights are quantized once before timing
+(fp4_quantize_weights, the load-time step).
+
+Workload: M=8192, N=28672, K=8192 (the large prefill GEMM), A ~ N(0,1) with
+0.1% of entries x100, W ~ N(0,0.02).  Inputs exceed L2 (A 128 MiB, packed W
+131 MiB, C 448 MiB), so no explicit flush is needed between steps.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun each rank runs an independent replica on its own GPU (the
+path has no exchange step); the value is total FLOPs over the max per-rank
+time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, N, K = 8192, 28672, 8192
+FLOP = 2.0 * M * N * K
+METRIC = "NVFP4 GEMM TFLOPS (% of B200 FP4 peak); quantize GB/s (% of HBM)"
+WORKLOAD = "prefill W4A4 NVFP4 GEMM M=8192 N=28672 K=8192, bf16 out, activation quantized per step"
+# algorithmic bytes per activation element of the DYNAMIC quantizer:
+# amax pass reads 2 B; quantize pass reads 2 B, writes 0.5 B codes + 1/16 B scales
+QUANT_BYTES_PER_ELEM = 2.0 + 2.0 + 0.5 + 1.0 / 16.0
+FP4_OVER_BF16 = 4.0     # nominal dense FP4 / dense BF16 tensor throughput on B200 (9 / 2.25)
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        busy = [s for s in sm if smax and s > 0.3 * smax] or sm
+        return {"sm_mhz": float(np.median(busy)) if busy else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(sample_rows=256, sample_cols=4096, seconds_target=10.0):
+    """The oracle, as it stands, on a bounded sample of the same workload:
+    quantize `sample_rows` rows of A and `sample_cols` rows of W (NVFP4,
+    global scales of the full tensors), dequantize, binary64 GEMM.  Returns
+    (TFLOP/s of the sampled GEMM incl. its quantization, threads, description)."""
+    import oracle
+    from mxfp4_block_scaled_fp4_b200 import inputs
+    g = inputs.rng(99, sample_rows, sample_cols, K)
+    a = inputs.to_bf16(inputs.normal(g, (sample_rows, K)))
+    w = inputs.to_bf16(inputs.normal(g, (sample_cols, K), 0.02))
+    oracle.lib()
+    reps, t_total = 0, 0.0
+    while t_total < seconds_target and reps < 50:
+        t0 = time.perf_counter()
+        ca, sa, ga = oracle.quantize_nvfp4(a)
+        cw, sw, gw = oracle.quantize_nvfp4(w)
+        oracle.gemm(oracle.dequant(ca, sa, 0, ga), oracle.dequant(cw, sw, 0, gw))
+        t_total += time.perf_counter() - t0
+        reps += 1
+    flop = 2.0 * sample_rows * sample_cols * K * reps
+    desc = (f"{sample_rows} rows of A x {sample_cols} rows of W at K={K} (NVFP4 quantize of "
+            f"both + binary64 GEMM), {reps} repetitions, {t_total:.1f} s")
+    return flop / t_total / 1e12, oracle.threads(), desc
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    val, cores, desc = cpu_baseline(seconds_target=max(5.0, 2.0 * (args.steps + args.warmup)))
+    line = {
+        "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": FLOP / (val * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "sample": desc},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    if args.warmup < 3:
+        args.warmup = 3
+
+    import torch
+    import torch.distributed as dist
+    from mxfp4_block_scaled_fp4_b200 import fp4lib as L, inputs, ops
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    L.lib()
+
+    a_cpu, w_cpu = inputs.prefill(M, N, K)
+    a = a_cpu.to(dev)
+    wq = ops.quantize_weights(w_cpu.to(dev), L.FP4_NVFP4)   # load-time step, untimed
+    del w_cpu
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(L.fp4_scale_bytes(M, K, 0, 0), dtype=torch.uint8, device=dev)
+    g_a = torch.empty(1, dtype=torch.float32, device=dev)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws_bytes = L.fp4_workspace_bytes(M, N, K, 0)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def check(st, what):
+        if st != 0:
+            raise L.Fp4Error(st, what)
+
+    ev_q0, ev_q1, ev_g1 = ([torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+                           for _ in range(3))
+
+    def step(i=None, timed=False):
+        if timed:
+            ev_q0[i].record(stream)
+        check(L.fp4_quantize_act(a.data_ptr(), M, K, 0, 0, 0, g_a.data_ptr(), codes.data_ptr(),
+                                 scales.data_ptr(), ws.data_ptr(), ws_bytes, sp), "quantize")
+        if timed:
+            ev_q1[i].record(stream)
+        check(L.fp4_gemm(codes.data_ptr(), scales.data_ptr(), g_a.data_ptr(), wq.codes.data_ptr(),
+                         wq.scales.data_ptr(), wq.g.data_ptr(), M, N, K, 0, c.data_ptr(), N, 0,
+                         ws.data_ptr(), ws_bytes, sp), "gemm")
+        if timed:
+            ev_g1[i].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, code = ops.device_status()
+    if st != 0:
+        raise RuntimeError(f"watchdog raised during warm-up: {code:#x}")
+
+    clocks = Clocks(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, timed=True)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    q_ms = float(np.mean([ev_q0[i].elapsed_time(ev_q1[i]) for i in range(args.steps)]))
+    g_ms = float(np.mean([ev_q1[i].elapsed_time(ev_g1[i]) for i in range(args.steps)]))
+    st, code = ops.device_status()
+    if st != 0:
+        raise RuntimeError(f"watchdog raised during timing: {code:#x}")
+
+    # ---- end to end through the C ABI with host buffers (pinned)
+    a_host = a_cpu.pin_memory()
+    c_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    e_steps = max(2, min(args.steps, 5))
+    for _ in range(2):
+        a.copy_(a_host, non_blocking=True)
+        step()
+        c_host.copy_(c, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        a.copy_(a_host, non_blocking=True)
+        step()
+        c_host.copy_(c, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+
+    times = torch.tensor([ms_total, e2e_ms, g_ms, q_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    ms_total, e2e_ms, g_ms, q_ms = times.tolist()
+    ms_step = ms_total / args.steps
+
+    peaks, src = load_peaks()
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
+    gemm_tflops = FLOP / (g_ms * 1e-3) / 1e12
+    q_bytes = QUANT_BYTES_PER_ELEM * M * K
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC,
+        "value": FLOP * world / (ms_step * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3 scales, fp32 accumulate, bf16 out)",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "format": "NVFP4",
+                   "global_scale": "dynamic", "out": "bf16",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (A 128 MiB, packed W 131 MiB, C 448 MiB)"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
+                     "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": None,
+                     "kernel": "fp4 gemm_kernel (tcgen05 kind::mxf4nvf4)",
+                     "peak_source": f"{src} bf16_tflops_sustained x {FP4_OVER_BF16:g} "
+                                    "(nominal dense FP4/BF16 ratio)"},
+        "quantize": {"achieved_gbs": q_gbs, "peak_gbs": peaks["hbm_gbs"],
+                     "frac": q_gbs / peaks["hbm_gbs"], "ms": q_ms,
+                     "bytes_per_elem": QUANT_BYTES_PER_ELEM,
+                     "note": "amax pass + quantize pass, algorithmic bytes (two reads of A)"},
+        "gemm_ms": g_ms,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+        "e2e": {"value": FLOP * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": a_host.numel() * 2, "d2h_bytes_per_step": c_host.numel() * 2},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, cores, desc = cpu_baseline()
+        line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,162 @@
+/*
+ * fp4.h -- C ABI of the B200 (sm_100a) W4A4 block-scaled FP4 library.
+ *
+ * Formats (sources are web pages, cited by title and section):
+ *  NVFP4  E2M1 codes {0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6}; every 16
+ *         consecutive values along K share an E4M3 scale chosen so the block
+ *         maximum lands on 6; a per-tensor FP32 global scale g keeps the
+ *         block scales inside E4M3's range (saturating, never NaN).
+ *         "Hardware FP4 inference for speech on Blackwell", section "NVFP4,
+ *         and the two ways it fails".
+ *  MXFP4  the OCP MX variant: 32 values per block share an E8M0 power-of-two
+ *         scale; no global scale.  "FP4 n'existe pas : il existe des FP4, et
+ *         chaque runtime choisit son dialecte", section "Deux dialectes, deux
+ *         strategies de scaling" and its format table.
+ *
+ * Operation (the W4A4 GEMM of the first page, "fp4-cuda-kernel" forum post:
+ * weights quantized once at load, activations quantized on the fly per call):
+ *     C[m, n] = alpha * sum_k  s_a[m, k/B] * q_a[m, k] * s_w[n, k/B] * q_w[n, k]
+ * with alpha = g_a * g_w (NVFP4) or 1 (MXFP4), accumulation in FP32.
+ *
+ * Conventions shared by every entry point
+ *  - Every pointer argument is a DEVICE pointer unless stated otherwise.
+ *    The caller allocates and owns all memory; the library never allocates,
+ *    frees or synchronizes (fp4_device_status is the one exception and says
+ *    so).  Work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and is asynchronous; global scales stay on the device.
+ *  - Argument checks happen before any launch and return a status; nothing
+ *    is enqueued when a check fails.  A failed launch returns FP4_ERR_CUDA.
+ *  - Shapes: rows (M or N) >= 0, K > 0 and K % 32 == 0 (a packed row of K/2
+ *    bytes must be a multiple of 16 bytes for the tensor-memory-accelerator
+ *    loads).  rows == 0 (or M == 0 / N == 0) is a no-op that returns FP4_OK
+ *    after the shape and enum checks, without looking at the pointers.
+ *    N % 8 == 0 for the GEMMs.
+ *  - Alignment: bf16 inputs, code and scale buffers and C are 16-byte
+ *    aligned; ldc * sizeof(element) is a multiple of 16; g pointers 4-byte.
+ *  - Packed codes: row-major [rows, K/2] bytes; element 2j of a row is the
+ *    low nibble of byte j, element 2j+1 the high nibble; a code is
+ *    sign<<3 | exponent<<1 | mantissa.
+ *  - Scales, FP4_SCALES_ROWMAJOR: [rows, K/B] bytes (B = 16 or 32).
+ *    FP4_SCALES_MMA: the order the tensor cores read.  Scales are grouped in
+ *    atoms of 128 rows x 4 scale columns (512 bytes); in an atom, row r and
+ *    column c sit at byte (r%32)*16 + (r/32)*4 + c; atom (rb, cb) starts at
+ *    byte (rb * ceil(nsf/4) + cb) * 512 with nsf = K/B.  Rows are padded to
+ *    a multiple of 128 and columns to a multiple of 4; the library writes
+ *    the padding as 0.
+ */
+#ifndef FP4_B200_H
+#define FP4_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP4_OK = 0,
+    FP4_ERR_INVALID_ARG = 1,        /* null pointer, bad enum, ldc < N, ... */
+    FP4_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 32 != 0, N % 8 != 0, negative size */
+    FP4_ERR_MISALIGNED = 3,         /* a pointer or leading dimension misaligned */
+    FP4_ERR_WORKSPACE_TOO_SMALL = 4,
+    FP4_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
+    FP4_ERR_DEVICE_TIMEOUT = 6,     /* a kernel's bounded wait ran out */
+    FP4_ERR_NO_DEVICE = 7           /* no sm_100 device is current */
+} fp4_status_t;
+
+typedef enum { FP4_NVFP4 = 0, FP4_MXFP4 = 1 } fp4_format_t;
+typedef enum { FP4_SCALES_MMA = 0, FP4_SCALES_ROWMAJOR = 1 } fp4_scale_layout_t;
+/* NVFP4 only: DYNAMIC computes g = amax(tensor) / 2688 on the device (g = 1
+ * for an all-zero tensor) and writes it to *g; STATIC reads a caller-chosen
+ * g from *g.  2688 = 6 * 448 ("Hardware FP4 inference for speech on
+ * Blackwell", section "NVFP4, and the two ways it fails"). */
+typedef enum { FP4_GLOBAL_DYNAMIC = 0, FP4_GLOBAL_STATIC = 1 } fp4_global_mode_t;
+typedef enum { FP4_OUT_BF16 = 0, FP4_OUT_F32 = 1 } fp4_out_t;
+
+/* Bytes of packed codes for a [rows, K] tensor: rows * K / 2. */
+size_t fp4_packed_bytes(int rows, int K);
+
+/* Bytes of scales for a [rows, K] tensor in the given layout (MMA layout
+ * includes its padding).  Returns 0 for an unsupported K. */
+size_t fp4_scale_bytes(int rows, int K, fp4_format_t fmt, fp4_scale_layout_t layout);
+
+/* Device workspace (bytes) that fp4_quantize_act / fp4_quantize_weights /
+ * fp4_gemm / fp4_gemm_fused need for a problem of this size.  The workspace
+ * holds per-block partial maxima of the DYNAMIC global-scale reduction and,
+ * for the small-M path, split-K partial sums; it needs no initialisation. */
+size_t fp4_workspace_bytes(int M, int N, int K, fp4_format_t fmt);
+
+/* Activation quantization, run per call: one pass of amax (DYNAMIC only) and
+ * one fused pass block-amax -> scale -> round-to-nearest-even to E2M1 ->
+ * nibble pack.  "Hardware FP4 inference for speech on Blackwell", section
+ * "NVFP4, and the two ways it fails" (s = E4M3(max|x|/6), x_hat = s*q, 448,
+ * 2688); MXFP4 per the format table of "FP4 n'existe pas".
+ *   x       bf16 [rows, K] row-major, contiguous
+ *   g       NVFP4: DYNAMIC writes g, STATIC reads g; MXFP4: ignored (may be NULL)
+ *   codes   [rows, K/2] bytes out; scales out in `layout`
+ *   ws      workspace of at least fp4_workspace_bytes(rows, 0, K, fmt) bytes
+ * Floating-point steps (one IEEE binary32 rounding each): g = amax/2688;
+ * sb = amax_b / (6 g); s = E4M3 round-to-nearest-even, saturating at 448;
+ * r = 1 / (s g); q = E2M1 round-to-nearest-even of x r, saturating at 6,
+ * sign kept (a negative value that rounds to zero is code 0x8); a block
+ * whose scale rounds to 0 gets all-zero codes.  MXFP4: e = floor(log2
+ * amax_b) - 2 clamped to [-127, 127], scale byte e + 127, q = E2M1(x 2^-e). */
+fp4_status_t fp4_quantize_act(const void* x, int rows, int K, fp4_format_t fmt,
+                              fp4_scale_layout_t layout, fp4_global_mode_t gmode,
+                              float* g, uint8_t* codes, uint8_t* scales,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* One-time weight quantization at load time ("fp4-cuda-kernel" forum post:
+ * quantize weights once at model load).  Same arithmetic as
+ * fp4_quantize_act with DYNAMIC global scale and scales written in the MMA
+ * layout.  w: bf16 [N, K]; g: NVFP4 out (may be NULL for MXFP4). */
+fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt,
+                                  uint8_t* codes, uint8_t* scales, float* g,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* Block-scaled FP4 GEMM on the tcgen05 tensor cores:
+ *     C[M, N] = alpha * A_hat[M, K] . W_hat[N, K]^T
+ * A and W are both K-major packed codes with MMA-layout scales (as written
+ * by the two quantizers above).  alpha = RN(g_a * g_w) for NVFP4 (g_a, g_w
+ * are device pointers) and 1 for MXFP4 (g_a, g_w may be NULL).  The sum is
+ * accumulated in FP32 in tensor memory; C = RN(alpha * acc) is written as
+ * bf16 (round to nearest even) or fp32, row-major with leading dimension
+ * ldc (elements).  Any M >= 0 (no padding asked of the caller), N % 8 == 0.
+ * The pages' W4A4 GEMM: "fp4-cuda-kernel" forum post; cuBLAS's refusal of
+ * M < 128 that this entry point does not share: "Hardware FP4 inference for
+ * speech on Blackwell", section "Do the FP4 tensor cores even engage?". */
+fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                      const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
+                      int M, int N, int K, fp4_format_t fmt,
+                      void* C, int ldc, fp4_out_t out,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Small-M path (decode): quantize the bf16 activation a [M, K] on the fly
+ * and multiply it with pre-quantized weights in one launch sequence, without
+ * a round trip of the quantized activation through global memory.
+ * "FP4 n'existe pas", runtime survey (quantization, scaling, matmul and
+ * de-scaling fused in one launch); the small-M regime: "Hardware FP4
+ * inference for speech on Blackwell", section "Do the FP4 tensor cores even
+ * engage?".  g_a: DYNAMIC writes it, STATIC reads it (NVFP4; MXFP4 ignores
+ * it).  Results equal fp4_quantize_act followed by fp4_gemm up to FP32
+ * summation order.  Requires M <= 32 (FP4_ERR_UNSUPPORTED_SHAPE otherwise). */
+fp4_status_t fp4_gemm_fused(const void* a, const uint8_t* w_codes, const uint8_t* w_scales,
+                            const float* g_w, int M, int N, int K, fp4_format_t fmt,
+                            fp4_global_mode_t gmode, float* g_a,
+                            void* C, int ldc, fp4_out_t out,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Reads and clears the device watchdog word that kernels set when one of
+ * their bounded waits runs out.  Synchronizes `stream`.  *code receives the
+ * raw word (0 = no timeout).  Returns FP4_ERR_DEVICE_TIMEOUT if it was set. */
+fp4_status_t fp4_device_status(unsigned* code, void* stream);
+
+/* A static string naming the status (never NULL). */
+const char* fp4_status_string(fp4_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4_B200_H */

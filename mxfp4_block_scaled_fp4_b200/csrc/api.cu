@@ -1,0 +1,241 @@
+// api.cu -- the extern "C" boundary: argument checks, workspace layout,
+// status strings.  Every computing step runs in the kernels of
+// quantize.cu, gemm.cu and fused.cu.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "fp4.h"
+#include "internal.h"
+
+namespace fp4 {
+
+// The watchdog word kernels set when a bounded wait runs out.
+static __device__ unsigned int g_watchdog = 0;
+
+unsigned* watchdog_ptr() {
+  static unsigned* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cached[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_watchdog) != cudaSuccess) return nullptr;
+    cached[dev] = static_cast<unsigned*>(p);
+  }
+  return cached[dev];
+}
+
+}  // namespace fp4
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+fp4_status_t check_format(fp4_format_t f) {
+  return (f == FP4_NVFP4 || f == FP4_MXFP4) ? FP4_OK : FP4_ERR_INVALID_ARG;
+}
+
+fp4_status_t check_rows_k(long long rows, int K) {
+  if (rows < 0 || K <= 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (K % 32 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+  return FP4_OK;
+}
+
+fp4_status_t device_ok() {
+  static int cached[64] = {0};   // 0 unknown, 1 ok, 2 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP4_ERR_NO_DEVICE;
+  if (cached[dev] == 0) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return FP4_ERR_NO_DEVICE;
+    cached[dev] = (major == 10) ? 1 : 2;
+  }
+  return cached[dev] == 1 ? FP4_OK : FP4_ERR_NO_DEVICE;
+}
+
+size_t quant_ws_bytes() { return static_cast<size_t>(fp4::kAmaxSlots) * sizeof(unsigned); }
+
+fp4_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t fp4_packed_bytes(int rows, int K) {
+  if (rows < 0 || K <= 0 || K % 2) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(K / 2);
+}
+
+size_t fp4_scale_bytes(int rows, int K, fp4_format_t fmt, fp4_scale_layout_t layout) {
+  if (check_format(fmt) != FP4_OK || check_rows_k(rows, K) != FP4_OK) return 0;
+  const int nsf = fp4::nsf_of(K, fmt);
+  if (layout == FP4_SCALES_ROWMAJOR) return static_cast<size_t>(rows) * nsf;
+  if (layout != FP4_SCALES_MMA) return 0;
+  return static_cast<size_t>((rows + 127) / 128) * fp4::ncb_of(nsf) * 512u;
+}
+
+size_t fp4_workspace_bytes(int M, int N, int K, fp4_format_t fmt) {
+  size_t w = quant_ws_bytes();
+  if (M > 0 && N > 0 && K > 0 && K % 32 == 0 && check_format(fmt) == FP4_OK) {
+    const size_t f = fp4::fused_workspace_bytes(M, N, K, fmt);
+    if (f > w) w = f;
+  }
+  return w;
+}
+
+fp4_status_t fp4_quantize_act(const void* x, int rows, int K, fp4_format_t fmt,
+                              fp4_scale_layout_t layout, fp4_global_mode_t gmode, float* g,
+                              uint8_t* codes, uint8_t* scales, void* ws, size_t ws_bytes,
+                              void* stream) {
+  fp4_status_t st;
+  if ((st = check_format(fmt)) != FP4_OK) return st;
+  if (layout != FP4_SCALES_MMA && layout != FP4_SCALES_ROWMAJOR) return FP4_ERR_INVALID_ARG;
+  if (gmode != FP4_GLOBAL_DYNAMIC && gmode != FP4_GLOBAL_STATIC) return FP4_ERR_INVALID_ARG;
+  if ((st = check_rows_k(rows, K)) != FP4_OK) return st;
+  if (rows == 0) return FP4_OK;   // nothing is read or written
+  const bool nv = fmt == FP4_NVFP4;
+  const bool dyn = nv && gmode == FP4_GLOBAL_DYNAMIC;
+  if (!x || !codes || !scales || (nv && !g) || (dyn && !ws)) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (nv && !aligned4(g)) ||
+      (dyn && !aligned16(ws)))
+    return FP4_ERR_MISALIGNED;
+  if (dyn && ws_bytes < quant_ws_bytes()) return FP4_ERR_WORKSPACE_TOO_SMALL;
+  if ((st = device_ok()) != FP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fp4::QuantArgs a{};
+  a.x = x;
+  a.rows = rows;
+  a.K = K;
+  a.fmt = fmt;
+  a.layout = layout;
+  a.dynamic = dyn ? 1 : 0;
+  a.g = g;
+  a.codes = codes;
+  a.scales = scales;
+  if (dyn) {
+    int used = 0;
+    unsigned* partial = static_cast<unsigned*>(ws);
+    if (fp4::launch_amax(x, static_cast<long long>(rows) * K, partial, &used, s) != cudaSuccess)
+      return FP4_ERR_CUDA;
+    a.partial = partial;
+    a.n_partial = used;
+  }
+  return from_cuda(fp4::launch_quantize(a, s));
+}
+
+fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt, uint8_t* codes,
+                                  uint8_t* scales, float* g, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  return fp4_quantize_act(w, N, K, fmt, FP4_SCALES_MMA, FP4_GLOBAL_DYNAMIC, g, codes, scales, ws,
+                          ws_bytes, stream);
+}
+
+fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                      const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, int M,
+                      int N, int K, fp4_format_t fmt, void* C, int ldc, fp4_out_t out, void* ws,
+                      size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  fp4_status_t st;
+  if ((st = check_format(fmt)) != FP4_OK) return st;
+  if (out != FP4_OUT_BF16 && out != FP4_OUT_F32) return FP4_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return FP4_OK;   // nothing is read or written
+  const bool nv = fmt == FP4_NVFP4;
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !C || (nv && (!g_a || !g_w)))
+    return FP4_ERR_INVALID_ARG;
+  if (ldc < N) return FP4_ERR_INVALID_ARG;
+  const int esize = out == FP4_OUT_F32 ? 4 : 2;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(C) || (static_cast<long long>(ldc) * esize) % 16 != 0 ||
+      (nv && (!aligned4(g_a) || !aligned4(g_w))))
+    return FP4_ERR_MISALIGNED;
+  if ((st = device_ok()) != FP4_OK) return st;
+  fp4::GemmArgs a{};
+  a.a_codes = a_codes;
+  a.a_scales = a_scales;
+  a.g_a = g_a;
+  a.w_codes = w_codes;
+  a.w_scales = w_scales;
+  a.g_w = g_w;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.fmt = fmt;
+  a.C = C;
+  a.ldc = ldc;
+  a.out_f32 = out == FP4_OUT_F32;
+  return from_cuda(fp4::launch_gemm(a, static_cast<cudaStream_t>(stream)));
+}
+
+fp4_status_t fp4_gemm_fused(const void* x, const uint8_t* w_codes, const uint8_t* w_scales,
+                            const float* g_w, int M, int N, int K, fp4_format_t fmt,
+                            fp4_global_mode_t gmode, float* g_a, void* C, int ldc, fp4_out_t out,
+                            void* ws, size_t ws_bytes, void* stream) {
+  fp4_status_t st;
+  if ((st = check_format(fmt)) != FP4_OK) return st;
+  if (out != FP4_OUT_BF16 && out != FP4_OUT_F32) return FP4_ERR_INVALID_ARG;
+  if (gmode != FP4_GLOBAL_DYNAMIC && gmode != FP4_GLOBAL_STATIC) return FP4_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (N % 8 != 0 || M > 32) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return FP4_OK;   // nothing is read or written
+  const bool nv = fmt == FP4_NVFP4;
+  if (!x || !w_codes || !w_scales || !C || !ws || (nv && (!g_a || !g_w)))
+    return FP4_ERR_INVALID_ARG;
+  if (ldc < N) return FP4_ERR_INVALID_ARG;
+  const int esize = out == FP4_OUT_F32 ? 4 : 2;
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(C) ||
+      !aligned16(ws) || (static_cast<long long>(ldc) * esize) % 16 != 0 ||
+      (nv && (!aligned4(g_a) || !aligned4(g_w))))
+    return FP4_ERR_MISALIGNED;
+  if (ws_bytes < fp4::fused_workspace_bytes(M, N, K, fmt)) return FP4_ERR_WORKSPACE_TOO_SMALL;
+  if ((st = device_ok()) != FP4_OK) return st;
+  fp4::FusedArgs a{};
+  a.a = x;
+  a.w_codes = w_codes;
+  a.w_scales = w_scales;
+  a.g_w = g_w;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.fmt = fmt;
+  a.dynamic = (nv && gmode == FP4_GLOBAL_DYNAMIC) ? 1 : 0;
+  a.g_a = g_a;
+  a.C = C;
+  a.ldc = ldc;
+  a.out_f32 = out == FP4_OUT_F32;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return from_cuda(fp4::launch_gemm_fused(a, static_cast<cudaStream_t>(stream)));
+}
+
+fp4_status_t fp4_device_status(unsigned* code, void* stream) {
+  if (!code) return FP4_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FP4_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, fp4::g_watchdog, sizeof v) != cudaSuccess) return FP4_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(fp4::g_watchdog, &zero, sizeof zero) != cudaSuccess)
+    return FP4_ERR_CUDA;
+  *code = v;
+  return v ? FP4_ERR_DEVICE_TIMEOUT : FP4_OK;
+}
+
+const char* fp4_status_string(fp4_status_t s) {
+  switch (s) {
+    case FP4_OK: return "ok";
+    case FP4_ERR_INVALID_ARG: return "invalid argument";
+    case FP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case FP4_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+    case FP4_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case FP4_ERR_CUDA: return "CUDA error";
+    case FP4_ERR_DEVICE_TIMEOUT: return "a device-side bounded wait timed out";
+    case FP4_ERR_NO_DEVICE: return "no sm_100 device is current";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

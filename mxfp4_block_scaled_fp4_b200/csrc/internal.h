@@ -1,0 +1,62 @@
+// internal.h -- launchers shared between the C-ABI layer and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace fp4 {
+
+constexpr int kAmaxSlots = 1024;   // partial maxima of the global-scale reduction
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count();
+
+// Device address of the watchdog word on the current device (cached per
+// device; nullptr if the symbol lookup fails).
+unsigned* watchdog_ptr();
+
+// Scale-layout geometry.
+inline int nsf_of(int K, int fmt) { return K / (fmt == 0 ? 16 : 32); }
+inline int ncb_of(int nsf) { return (nsf + 3) / 4; }
+inline long long rows_pad128(long long rows) { return (rows + 127) / 128 * 128; }
+
+// amax over a bf16 tensor of n elements (n % 8 == 0): writes one partial
+// maximum (bf16 magnitude bits) per CTA into `partial`; *n_used = CTAs.
+cudaError_t launch_amax(const void* x, long long n, unsigned* partial, int* n_used,
+                        cudaStream_t s);
+
+struct QuantArgs {
+  const void* x;        // bf16 [rows, K]
+  long long rows;
+  int K;
+  int fmt;              // 0 NVFP4, 1 MXFP4
+  int layout;           // 0 MMA, 1 row-major
+  int dynamic;          // NVFP4: 1 = g from partial maxima, 0 = read *g
+  float* g;
+  const unsigned* partial;
+  int n_partial;
+  uint8_t* codes;
+  uint8_t* scales;
+};
+cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s);
+
+struct GemmArgs {
+  const uint8_t* a_codes; const uint8_t* a_scales; const float* g_a;
+  const uint8_t* w_codes; const uint8_t* w_scales; const float* g_w;
+  int M, N, K, fmt;
+  void* C; int ldc; int out_f32;
+};
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s);
+
+struct FusedArgs {
+  const void* a;        // bf16 [M, K]
+  const uint8_t* w_codes; const uint8_t* w_scales; const float* g_w;
+  int M, N, K, fmt, dynamic;
+  float* g_a;
+  void* C; int ldc; int out_f32;
+  void* ws; size_t ws_bytes;
+};
+size_t fused_workspace_bytes(int M, int N, int K, int fmt);
+cudaError_t launch_gemm_fused(const FusedArgs& a, cudaStream_t s);
+
+}  // namespace fp4

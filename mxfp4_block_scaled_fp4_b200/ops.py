@@ -1,0 +1,134 @@
+"""Torch-facing wrappers over the C ABI.
+
+PyTorch is only the plumbing here: it allocates device memory and supplies
+the current CUDA stream.  Each function checks its tensors, allocates the
+outputs and calls one C entry point; the work runs in the library's kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import fp4lib as L
+
+NVFP4 = L.FP4_NVFP4
+MXFP4 = L.FP4_MXFP4
+SCALES_MMA = L.FP4_SCALES_MMA
+SCALES_ROWMAJOR = L.FP4_SCALES_ROWMAJOR
+
+_ws_cache: dict[int, torch.Tensor] = {}
+
+
+def workspace(nbytes: int, device: torch.device) -> torch.Tensor:
+    """A grow-only per-device scratch buffer (no initialisation needed)."""
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    buf = _ws_cache.get(idx)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 1 << 16), dtype=torch.uint8, device=device)
+        _ws_cache[idx] = buf
+    return buf
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(status: int, what: str):
+    if status != L.FP4_OK:
+        raise L.Fp4Error(status, what)
+
+
+def _cuda_bf16_2d(t: torch.Tensor, name: str):
+    if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous 2-D bf16 CUDA tensor")
+
+
+@dataclass
+class Quantized:
+    """Packed FP4 codes + scales + global scale of a [rows, K] tensor."""
+    codes: torch.Tensor      # uint8 [rows, K/2]
+    scales: torch.Tensor     # uint8, layout-dependent size
+    g: torch.Tensor          # float32 [1] (NVFP4); ones for MXFP4
+    fmt: int
+    layout: int
+    rows: int
+    K: int
+
+
+def quantize(x: torch.Tensor, fmt: int = NVFP4, layout: int = SCALES_MMA,
+             g: torch.Tensor | None = None) -> Quantized:
+    """fp4_quantize_act: DYNAMIC global scale when g is None, else STATIC g."""
+    _cuda_bf16_2d(x, "x")
+    rows, K = x.shape
+    dev = x.device
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(max(L.fp4_scale_bytes(rows, K, fmt, layout), 1), dtype=torch.uint8,
+                         device=dev)
+    gmode = L.FP4_GLOBAL_DYNAMIC if g is None else L.FP4_GLOBAL_STATIC
+    gt = torch.ones(1, dtype=torch.float32, device=dev) if g is None else g
+    ws_bytes = L.fp4_workspace_bytes(rows, 0, K, fmt)
+    ws = workspace(ws_bytes, dev)
+    _check(L.fp4_quantize_act(x.data_ptr(), rows, K, fmt, layout, gmode, gt.data_ptr(),
+                              codes.data_ptr(), scales.data_ptr(), ws.data_ptr(), ws.numel(),
+                              _stream()), "fp4_quantize_act")
+    return Quantized(codes, scales, gt, fmt, layout, rows, K)
+
+
+def quantize_weights(w: torch.Tensor, fmt: int = NVFP4) -> Quantized:
+    """fp4_quantize_weights: one-time, MMA scale layout, DYNAMIC g."""
+    _cuda_bf16_2d(w, "w")
+    N, K = w.shape
+    dev = w.device
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(max(L.fp4_scale_bytes(N, K, fmt, SCALES_MMA), 1), dtype=torch.uint8,
+                         device=dev)
+    g = torch.ones(1, dtype=torch.float32, device=dev)
+    ws = workspace(L.fp4_workspace_bytes(N, 0, K, fmt), dev)
+    _check(L.fp4_quantize_weights(w.data_ptr(), N, K, fmt, codes.data_ptr(), scales.data_ptr(),
+                                  g.data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
+           "fp4_quantize_weights")
+    return Quantized(codes, scales, g, fmt, SCALES_MMA, N, K)
+
+
+def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
+         out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp4_gemm: C = alpha * A_hat . W_hat^T."""
+    if a.fmt != w.fmt or a.K != w.K or a.layout != SCALES_MMA or w.layout != SCALES_MMA:
+        raise ValueError("operands must share format and K and use the MMA scale layout")
+    M, N, K = a.rows, w.rows, a.K
+    dev = a.codes.device
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    o = L.FP4_OUT_F32 if out.dtype == torch.float32 else L.FP4_OUT_BF16
+    _check(L.fp4_gemm(a.codes.data_ptr(), a.scales.data_ptr(), a.g.data_ptr(),
+                      w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(), M, N, K, a.fmt,
+                      out.data_ptr(), out.stride(0), o, None, 0, _stream()), "fp4_gemm")
+    return out
+
+
+def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
+               g_a: torch.Tensor | None = None, out: torch.Tensor | None = None,
+               g_out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp4_gemm_fused: quantize x (M <= 32) on the fly and multiply with w."""
+    _cuda_bf16_2d(x, "x")
+    M, K = x.shape
+    N = w.rows
+    dev = x.device
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    o = L.FP4_OUT_F32 if out.dtype == torch.float32 else L.FP4_OUT_BF16
+    gmode = L.FP4_GLOBAL_DYNAMIC if g_a is None else L.FP4_GLOBAL_STATIC
+    if g_a is None:
+        g_a = g_out if g_out is not None else torch.ones(1, dtype=torch.float32, device=dev)
+    ws = workspace(L.fp4_workspace_bytes(M, N, K, w.fmt), dev)
+    _check(L.fp4_gemm_fused(x.data_ptr(), w.codes.data_ptr(), w.scales.data_ptr(),
+                            w.g.data_ptr(), M, N, K, w.fmt, gmode, g_a.data_ptr(),
+                            out.data_ptr(), out.stride(0), o, ws.data_ptr(), ws.numel(),
+                            _stream()), "fp4_gemm_fused")
+    return out
+
+
+def device_status():
+    """(status, watchdog word); synchronizes the current stream."""
+    return L.fp4_device_status(_stream())

@@ -1,0 +1,91 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and its host-only functions (sizes, argument checks, status
+strings) behave as documented.  No compute call is made here."""
+import ctypes
+
+import pytest
+
+from mxfp4_block_scaled_fp4_b200 import fp4lib as L
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mxfp4_block_scaled_fp4_b200 import build
+    build.build()
+    return L.lib()
+
+
+def test_exports_every_header_symbol(lib):
+    names = L.header_symbols()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in L.SIGNATURES, n
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert L.fp4_status_string(s)
+    assert L.fp4_status_string(0) == "ok"
+    assert L.fp4_status_string(99) == "unknown status"
+
+
+def test_size_queries(lib):
+    assert L.fp4_packed_bytes(16, 256) == 16 * 128
+    assert L.fp4_scale_bytes(16, 256, L.FP4_NVFP4, L.FP4_SCALES_ROWMAJOR) == 16 * 16
+    assert L.fp4_scale_bytes(16, 256, L.FP4_MXFP4, L.FP4_SCALES_ROWMAJOR) == 16 * 8
+    # MMA order: rows padded to 128, scale columns to multiples of 4 (512-byte atoms)
+    assert L.fp4_scale_bytes(16, 256, L.FP4_NVFP4, L.FP4_SCALES_MMA) == 4 * 512
+    assert L.fp4_scale_bytes(130, 2880, L.FP4_NVFP4, L.FP4_SCALES_MMA) == 2 * 45 * 512
+    assert L.fp4_scale_bytes(1, 2880, L.FP4_MXFP4, L.FP4_SCALES_MMA) == 23 * 512
+    assert L.fp4_scale_bytes(4, 100, L.FP4_NVFP4, L.FP4_SCALES_MMA) == 0     # K % 32
+    assert L.fp4_workspace_bytes(8192, 0, 16384, L.FP4_NVFP4) >= 4096
+
+
+def test_scale_bytes_match_oracle_layout(lib, orc):
+    for rows, K in [(1, 256), (16, 2880), (300, 8192)]:
+        assert L.fp4_scale_bytes(rows, K, L.FP4_NVFP4, L.FP4_SCALES_MMA) == \
+            orc.mma_scale_bytes(rows, K // 16)
+        assert L.fp4_scale_bytes(rows, K, L.FP4_MXFP4, L.FP4_SCALES_MMA) == \
+            orc.mma_scale_bytes(rows, K // 32)
+
+
+def test_argument_checks_fail_before_any_launch(lib):
+    fake = ctypes.c_void_p(1 << 20)           # never dereferenced: checks fail first
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    q = L.fp4_quantize_act
+    assert q(fake, 4, 100, 0, 0, 0, fake, fake, fake, fake, 1 << 16, None) == \
+        L.FP4_ERR_UNSUPPORTED_SHAPE
+    assert q(fake, -1, 256, 0, 0, 0, fake, fake, fake, fake, 1 << 16, None) == \
+        L.FP4_ERR_UNSUPPORTED_SHAPE
+    assert q(None, 4, 256, 0, 0, 0, fake, fake, fake, fake, 1 << 16, None) == \
+        L.FP4_ERR_INVALID_ARG
+    assert q(fake, 4, 256, 7, 0, 0, fake, fake, fake, fake, 1 << 16, None) == \
+        L.FP4_ERR_INVALID_ARG
+    assert q(mis, 4, 256, 0, 0, 0, fake, fake, fake, fake, 1 << 16, None) == \
+        L.FP4_ERR_MISALIGNED
+    assert q(fake, 4, 256, 0, 0, 0, fake, fake, fake, fake, 16, None) == \
+        L.FP4_ERR_WORKSPACE_TOO_SMALL
+    g = L.fp4_gemm
+    assert g(fake, fake, fake, fake, fake, fake, 4, 12, 256, 0, fake, 12, 0, None, 0, None) == \
+        L.FP4_ERR_UNSUPPORTED_SHAPE                                   # N % 8
+    assert g(fake, fake, fake, fake, fake, fake, 4, 16, 256, 0, fake, 8, 0, None, 0, None) == \
+        L.FP4_ERR_INVALID_ARG                                         # ldc < N
+    assert g(fake, fake, fake, fake, fake, fake, 4, 16, 256, 0, fake, 20, 0, None, 0, None) == \
+        L.FP4_ERR_MISALIGNED                                          # ldc*2 % 16
+    assert g(fake, fake, None, fake, fake, fake, 4, 16, 256, 0, fake, 16, 0, None, 0, None) == \
+        L.FP4_ERR_INVALID_ARG                                         # NVFP4 needs g_a
+    f = L.fp4_gemm_fused
+    assert f(fake, fake, fake, fake, 33, 16, 256, 0, 0, fake, fake, 16, 0, fake, 1 << 30, None) == \
+        L.FP4_ERR_UNSUPPORTED_SHAPE                                   # M > 32
+    assert f(fake, fake, fake, fake, 8, 16, 256, 0, 0, fake, fake, 16, 0, fake, 16, None) == \
+        L.FP4_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_no_gpu_means_no_device_status(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    fake = ctypes.c_void_p(1 << 20)
+    st = L.fp4_quantize_act(fake, 4, 256, 0, 0, 0, fake, fake, fake, fake, 1 << 16, None)
+    assert st in (L.FP4_ERR_NO_DEVICE,)

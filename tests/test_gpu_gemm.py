@@ -1,0 +1,99 @@
+"""GPU W4A4 GEMM (quantize on the GPU, tcgen05 GEMM) against the oracle's
+binary64 product of its own dequantized operands, within the stated
+tolerance (tests/parity.py), on the tiny outlier problem, ragged shapes
+that span several tiles and a K tail, the decode shapes through the fused
+entry point, and sampled outputs of the full-size prefill shapes."""
+import numpy as np
+import pytest
+import torch
+
+from mxfp4_block_scaled_fp4_b200 import inputs
+from tests.parity import bits, gemm_close
+
+pytestmark = pytest.mark.gpu
+DT = {"bf16": torch.bfloat16, "f32": torch.float32}
+
+
+@pytest.fixture(scope="module")
+def ops():
+    from mxfp4_block_scaled_fp4_b200 import ops as o
+    return o
+
+
+def run_pair(ops, orc, a, w, fmt, dt, fused=False):
+    aq_ref = orc.quantize(a, fmt)
+    wq_ref = orc.quantize(w, fmt)
+    c_ref = orc.gemm(orc.dequant(aq_ref[0], aq_ref[1], fmt, aq_ref[2]),
+                     orc.dequant(wq_ref[0], wq_ref[1], fmt, wq_ref[2]))
+    wq = ops.quantize_weights(w.cuda(), fmt)
+    if fused:
+        g_out = torch.zeros(1, dtype=torch.float32, device="cuda")
+        c = ops.gemm_fused(a.cuda(), wq, DT[dt], g_out=g_out)
+    else:
+        aq = ops.quantize(a.cuda(), fmt, ops.SCALES_MMA)
+        c = ops.gemm(aq, wq, DT[dt])
+    torch.cuda.synchronize()
+    st, code = ops.device_status()
+    assert st == 0 and code == 0
+    assert np.array_equal(bits(wq.codes), wq_ref[0])
+    ok, worst, where = gemm_close(c, c_ref, DT[dt])
+    assert ok, f"worst err/bound {worst:.3g} at {where}"
+    if fused and fmt == 0:
+        assert np.float32(g_out.item()).tobytes() == np.float32(aq_ref[2]).tobytes()
+    return c, c_ref
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("fused", [False, True])
+def test_pr1_tiny_outliers(ops, orc, fmt, dt, fused):
+    a, w = inputs.pr1_tiny()
+    run_pair(ops, orc, a, w, fmt, dt, fused)
+
+
+RAGGED = [(1, 8, 32), (16, 256, 64), (130, 264, 2880), (300, 520, 1056), (257, 512, 4096),
+          (128, 256, 256), (129, 136, 96)]
+
+
+@pytest.mark.parametrize("M,N,K", RAGGED)
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_ragged_shapes(ops, orc, M, N, K, fmt, dt):
+    a = inputs.random_bf16(100 + M, (M, K))
+    w = inputs.random_bf16(200 + N, (N, K), 0.02)
+    run_pair(ops, orc, a, w, fmt, dt)
+
+
+@pytest.mark.parametrize("M", [1, 8, 32])
+@pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096), (4096, 14336)])
+def test_decode_shapes_fused(ops, orc, M, N, K):
+    a, w = inputs.decode(M, N, K)
+    run_pair(ops, orc, a, w, 0, "bf16", fused=True)
+
+
+@pytest.mark.parametrize("M,N,K,fmt,dt", [(8192, 28672, 8192, 0, "bf16"),
+                                          (2048, 8192, 8192, 0, "f32"),
+                                          (2048, 8192, 8192, 1, "bf16")])
+def test_prefill_full_size_sampled(ops, orc, M, N, K, fmt, dt):
+    """Full-size launch; the oracle computes 128 sampled rows x 128 sampled
+    columns (each row quantized with the tensor's own global scale)."""
+    a, w = inputs.prefill(M, N, K)
+    wq = ops.quantize_weights(w.cuda(), fmt)
+    aq = ops.quantize(a.cuda(), fmt, ops.SCALES_MMA)
+    c = ops.gemm(aq, wq, DT[dt])
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(M + N)
+    ri = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 126, replace=False)]))
+    ci = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 126, replace=False)]))
+    g_a = orc.global_scale(orc.amax(a)) if fmt == 0 else None
+    g_w = orc.global_scale(orc.amax(w)) if fmt == 0 else None
+    if fmt == 0:
+        assert np.float32(aq.g.item()).tobytes() == np.float32(g_a).tobytes()
+        assert np.float32(wq.g.item()).tobytes() == np.float32(g_w).tobytes()
+    rt, ct = torch.from_numpy(ri), torch.from_numpy(ci)
+    ca, sa, ga = orc.quantize(a[rt].contiguous(), fmt, g_a)
+    cw, sw, gw = orc.quantize(w[ct].contiguous(), fmt, g_w)
+    assert np.array_equal(bits(aq.codes[rt.cuda()]), ca)
+    c_ref = orc.gemm(orc.dequant(ca, sa, fmt, ga), orc.dequant(cw, sw, fmt, gw))
+    ok, worst, where = gemm_close(c[rt.cuda()][:, ct.cuda()], c_ref, DT[dt])
+    assert ok, f"worst err/bound {worst:.3g} at {where}"
