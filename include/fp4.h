@@ -147,6 +147,32 @@ fp4_status_t fp4_gemm_fused(const void* a, const uint8_t* w_codes, const uint8_t
                             void* C, int ldc, fp4_out_t out,
                             void* ws, size_t ws_bytes, void* stream);
 
+/* Activation quantization without a workspace argument, for callers that
+ * cannot allocate device memory: code running while a stream is captured
+ * into a CUDA graph (a cudaMalloc there breaks the capture), engines that
+ * reserve all device memory at start-up and allow no later allocation, and
+ * latency-critical paths that cannot pay for cudaMalloc's implicit
+ * synchronization.  The pages have no counterpart of this entry point.
+ * Same arguments (minus ws / ws_bytes), arithmetic and results as
+ * fp4_quantize_act.  The DYNAMIC global-scale reduction keeps its partial
+ * maxima in a fixed 4 KiB device array inside the library instead of a
+ * caller workspace; the array exists on every GPU that loads the library
+ * until the process exits.  Limit: the call is rejected with
+ * FP4_ERR_WORKSPACE_TOO_SMALL if the scratch it needs
+ * (fp4_workspace_bytes(rows, 0, K, fmt)) exceeds those 4 KiB; today that
+ * need is 4 KiB for every accepted size.  The first DYNAMIC call on a device
+ * looks up the array's device address (cudaGetSymbolAddress, once per
+ * device); make that first call before any stream capture.  All calls share
+ * the array: calls that overlap on the GPU (other streams, other host
+ * threads on the same device) race and must not be issued.  The array keeps
+ * the last call's contents; no clearing is needed since every call writes
+ * each slot before reading it.  No cudaMalloc / cudaFree or other allocating
+ * call is made. */
+fp4_status_t fp4_quantize_act_noalloc(const void* x, int rows, int K, fp4_format_t fmt,
+                                      fp4_scale_layout_t layout, fp4_global_mode_t gmode,
+                                      float* g, uint8_t* codes, uint8_t* scales,
+                                      void* stream);
+
 /* Reads and clears the device watchdog word that kernels set when one of
  * their bounded waits runs out.  Synchronizes `stream`.  *code receives the
  * raw word (0 = no timeout).  Returns FP4_ERR_DEVICE_TIMEOUT if it was set. */

@@ -60,6 +60,7 @@ SIGNATURES = {
     "fp4_quantize_weights": (I, [P, I, I, I, U8P, U8P, FP, P, SZ, P]),
     "fp4_gemm": (I, [U8P, U8P, FP, U8P, U8P, FP, I, I, I, I, P, I, I, P, SZ, P]),
     "fp4_gemm_fused": (I, [P, U8P, U8P, FP, I, I, I, I, I, FP, P, I, I, P, SZ, P]),
+    "fp4_quantize_act_noalloc": (I, [P, I, I, I, I, I, FP, U8P, U8P, P]),
     "fp4_device_status": (I, [ctypes.POINTER(ctypes.c_uint), P]),
     "fp4_status_string": (ctypes.c_char_p, [I]),
 }
@@ -125,6 +126,11 @@ def fp4_gemm_fused(a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc, 
                    ws_bytes, stream):
     return _call("fp4_gemm_fused", a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc,
                  out, ws, ws_bytes, stream)
+
+
+def fp4_quantize_act_noalloc(x, rows, K, fmt, layout, gmode, g, codes, scales, stream):
+    return _call("fp4_quantize_act_noalloc", x, rows, K, fmt, layout, gmode, g, codes, scales,
+                 stream)
 
 
 def fp4_device_status(stream=None):
