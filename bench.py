@@ -128,7 +128,7 @@ def cpu_baseline(sample_rows=256, sample_cols=4096, seconds_target=10.0):
 def run_reference(args, rank):
     if rank != 0:
         return 0
-    val, cores, desc = cpu_baseline(seconds_target=max(5.0, 2.0 * (args.steps + args.warmup)))
+    val, cores, desc = cpu_baseline(seconds_target=min(20.0, max(5.0, 0.5 * (args.steps + args.warmup))))
     line = {
         "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": FLOP / (val * 1e12) * 1e3,
@@ -150,7 +150,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default=None,
+                    help="M,N,K override (profiling of smaller cases); default 8192,28672,8192")
     args = ap.parse_args()
+    if args.shape:
+        global M, N, K, FLOP, WORKLOAD
+        M, N, K = (int(v) for v in args.shape.split(","))
+        FLOP = 2.0 * M * N * K
+        WORKLOAD = (f"W4A4 NVFP4 GEMM M={M} N={N} K={K}, bf16 out, activation quantized per step"
+                    " (profiling shape)")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
