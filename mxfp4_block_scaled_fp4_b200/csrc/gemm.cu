@@ -13,13 +13,20 @@
 //               row, 128-byte swizzle) and the matching scale atoms (plain
 //               bulk copies: in the MMA scale order a tile's scales for one
 //               K step are contiguous) into a 4-stage shared-memory ring;
-//   warp 1      one thread issues tcgen05.cp (scales: shared -> tensor
-//               memory) and tcgen05.mma kind::mxf4nvf4 (128 x 256 x 64 per
-//               instruction) into an FP32 accumulator in tensor memory, and
-//               releases ring stages with tcgen05.commit;
+//   warp 1      one thread issues tcgen05.mma kind::mxf4nvf4 (128 x 256 x 64
+//               per instruction) into an FP32 accumulator in tensor memory
+//               and releases ring stages with tcgen05.commit;
 //   warps 2-5   epilogue: tcgen05.ld the accumulator (one 32-lane quarter
 //               per warp), multiply by alpha, round to bf16 / keep fp32,
-//               store C.
+//               store C;
+//   warps 6-9   scale staging: each warp reads a stage's scale atoms from
+//               shared memory and writes them with tcgen05.st into its own
+//               32-lane quarter of the stage's scale region in tensor memory
+//               (every quarter gets the whole 32-row x 16-byte block of an
+//               atom, the image the MMA reads), then signals the MMA thread.
+//               Moving scales with warp stores instead of tcgen05.cp keeps
+//               the copies out of the MMA pipe: measured on B200, even one
+//               tcgen05.cp per K step stalled the MMAs of every step.
 // Every mbarrier wait is bounded; a wait that runs out sets the watchdog
 // word, the CTA stops issuing, waits (bounded) for its copies and MMAs in
 // flight, frees its tensor memory and returns.
@@ -45,12 +52,12 @@ constexpr int B_STAGE = BN * BK_BYTES;  // 32 KiB
 constexpr int SFA_STAGE = 4 * 512;      // up to 4 scale atoms (128 rows x 4 scales)
 constexpr int SFB_STAGE = 2 * 4 * 512;  // two 128-row blocks x 4 atoms
 constexpr int RING_BYTES = STAGES * (A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE);
-constexpr int SMEM_BYTES = RING_BYTES + 1024 + 256;
+constexpr int SMEM_BYTES = RING_BYTES + 1024 + 256;   // ring + alignment + barriers
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;         // 256 fp32 columns
 constexpr uint32_t SF_COL = 256;        // per stage: 16 columns A scales + 32 B scales
 constexpr uint32_t SF_STAGE_COLS = 48;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;       // 10 warps: TMA, MMA, 4 epilogue, 4 scale staging
 constexpr int GROUP_M = 16;             // tile raster: 16 M-tiles share their W tiles in L2
 
 struct Params {
@@ -90,7 +97,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* sSFB = sSFA + STAGES * SFA_STAGE;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_STAGE);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
+  uint64_t* sf_full = empty + STAGES;
+  uint64_t* acc_full = sf_full + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -103,6 +111,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], 4);   // one arrival per scale-staging warp
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);   // one arrival per epilogue warp
@@ -175,22 +184,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         goto mma_drain;
       tc_fence_after();
       for (int kb = 0; kb < p.k_steps; ++kb) {
+        // the staging warps consumed full[stage] before arriving on sf_full[stage]
         if (!mbar_wait(&full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) goto mma_drain;
+        if (!mbar_wait(&sf_full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) goto mma_drain;
         tc_fence_after();
         {
-          const int cb0 = kb * kAtomsPerStage;
-          const int atoms = min(kAtomsPerStage, p.ncb - cb0);
           const int n_mma = min(BK / MMA_K, (p.K - kb * BK + MMA_K - 1) / MMA_K);
           const uint32_t sfa_t = tmem + SF_COL + stage * SF_STAGE_COLS;
           const uint32_t sfb_t = sfa_t + 16;
-          const uint32_t sfa_s = smem_u32(sSFA + stage * SFA_STAGE);
-          const uint32_t sfb_s = smem_u32(sSFB + stage * SFB_STAGE);
-          for (int a = 0; a < atoms; ++a) {
-            tc_cp_32x128b_x4(sfa_t + 4 * a, smem_desc(sfa_s + a * 512, 16, 128, kLayoutNone));
-            tc_cp_32x128b_x4(sfb_t + 8 * a, smem_desc(sfb_s + a * 512, 16, 128, kLayoutNone));
-            tc_cp_32x128b_x4(sfb_t + 8 * a + 4,
-                             smem_desc(sfb_s + 2048 + a * 512, 16, 128, kLayoutNone));
-          }
           const uint32_t a_s = smem_u32(sA + stage * A_STAGE);
           const uint32_t b_s = smem_u32(sB + stage * B_STAGE);
           for (int k = 0; k < n_mma; ++k) {
@@ -220,6 +221,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_commit(drain);
     mbar_wait_drain(drain, 0, p.watchdog);
   mma_done:;
+  } else if (warp >= 6) {
+    // ----------------------------------------------------- scale staging
+    const int quarter = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < n_tiles_total; t += gridDim.x) {
+      for (int kb = 0; kb < p.k_steps; ++kb) {
+        // warp-uniform outcome: tcgen05.st below needs all 32 lanes
+        if (!__all_sync(0xFFFFFFFFu,
+                        mbar_wait(&full[stage], phase, abort_flag, p.watchdog, WD_STAGING)))
+          goto staging_done;
+        {
+          const uint32_t sfa_s = smem_u32(sSFA + stage * SFA_STAGE) + lane * 16;
+          const uint32_t sfb_s = smem_u32(sSFB + stage * SFB_STAGE) + lane * 16;
+          const uint32_t sfa_t = tmem + lane_off + SF_COL + stage * SF_STAGE_COLS;
+          const uint32_t sfb_t = sfa_t + 16;
+          // atom a, row `lane`: 16 bytes = 4 columns; A at columns 4a..4a+3,
+          // W row block rb at columns 8a + 4rb .. 8a + 4rb + 3
+          uint32_t va[4 * kAtomsPerStage], vb[8 * kAtomsPerStage];
+#pragma unroll
+          for (int a = 0; a < kAtomsPerStage; ++a) {
+            const uint4 x = lds128(sfa_s + a * 512);
+            va[4 * a + 0] = x.x; va[4 * a + 1] = x.y; va[4 * a + 2] = x.z; va[4 * a + 3] = x.w;
+#pragma unroll
+            for (int rb = 0; rb < 2; ++rb) {
+              const uint4 y = lds128(sfb_s + rb * 2048 + a * 512);
+              vb[8 * a + 4 * rb + 0] = y.x; vb[8 * a + 4 * rb + 1] = y.y;
+              vb[8 * a + 4 * rb + 2] = y.z; vb[8 * a + 4 * rb + 3] = y.w;
+            }
+          }
+          if (kAtomsPerStage == 4) {
+            tmem_st_x16(sfa_t, va);
+            tmem_st_x32(sfb_t, vb);
+          } else {
+            tmem_st_x8(sfa_t, va);
+            tmem_st_x16(sfb_t, vb);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  staging_done:;
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;        // tensor-memory lanes this warp may read
@@ -229,7 +280,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int t = blockIdx.x; t < n_tiles_total; t += gridDim.x, ++it) {
       int mt, nt;
       tile_coords(t, p, mt, nt);
-      if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag, p.watchdog, WD_EPILOGUE)) break;
+      // warp-uniform outcome: tcgen05.ld below needs all 32 lanes
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag,
+                                             p.watchdog, WD_EPILOGUE)))
+        break;
       tc_fence_after();
       const int row = mt * BM + quarter * 32 + lane;
       const bool row_ok = row < p.M;
