@@ -97,7 +97,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* sSFB = sSFA + STAGES * SFA_STAGE;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_STAGE);
   uint64_t* empty = full + STAGES;
-  uint64_t* sf_full = empty + STAGES;
+  uint64_t* sf_loaded = empty + STAGES;
+  uint64_t* sf_full = sf_loaded + STAGES;
   uint64_t* acc_full = sf_full + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_loaded[s], 1);
       mbar_init(&sf_full[s], 4);   // one arrival per scale-staging warp
     }
     mbar_init(acc_full, 1);
@@ -149,16 +151,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
           const int rb0 = nt * 2;
           const int wblocks = min(2, p.w_rowblocks - rb0);
-          mbar_expect_tx(&full[stage], A_STAGE + B_STAGE + sf_bytes * (1 + wblocks));
-          tma_load_2d(sA + stage * A_STAGE, &tm_a, kb * BK_BYTES, mt * BM, &full[stage]);
-          tma_load_2d(sB + stage * B_STAGE, &tm_w, kb * BK_BYTES, nt * BN, &full[stage]);
+          // scales first, on their own barrier, so that staging them into
+          // tensor memory overlaps the (larger) code tiles' flight
+          mbar_expect_tx(&sf_loaded[stage], sf_bytes * (1 + wblocks));
           bulk_load(sSFA + stage * SFA_STAGE,
                     p.a_scales + (static_cast<long long>(mt) * p.ncb + cb0) * 512, sf_bytes,
-                    &full[stage]);
+                    &sf_loaded[stage]);
           for (int i = 0; i < wblocks; ++i)
             bulk_load(sSFB + stage * SFB_STAGE + i * 2048,
                       p.w_scales + (static_cast<long long>(rb0 + i) * p.ncb + cb0) * 512, sf_bytes,
-                      &full[stage]);
+                      &sf_loaded[stage]);
+          mbar_expect_tx(&full[stage], A_STAGE + B_STAGE);
+          tma_load_2d(sA + stage * A_STAGE, &tm_a, kb * BK_BYTES, mt * BM, &full[stage]);
+          tma_load_2d(sB + stage * B_STAGE, &tm_w, kb * BK_BYTES, nt * BN, &full[stage]);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         }
@@ -172,7 +177,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   producer_drain:
     // let every copy this thread started land before the CTA goes away
     for (int s = 0; s < STAGES; ++s)
-      if (armed & (1u << s)) mbar_wait_drain(&full[s], (armed_parity >> s) & 1u, p.watchdog);
+      if (armed & (1u << s)) {
+        mbar_wait_drain(&sf_loaded[s], (armed_parity >> s) & 1u, p.watchdog);
+        mbar_wait_drain(&full[s], (armed_parity >> s) & 1u, p.watchdog);
+      }
   producer_done:;
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------- MMA issuer
@@ -184,7 +192,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         goto mma_drain;
       tc_fence_after();
       for (int kb = 0; kb < p.k_steps; ++kb) {
-        // the staging warps consumed full[stage] before arriving on sf_full[stage]
         if (!mbar_wait(&full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) goto mma_drain;
         if (!mbar_wait(&sf_full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) goto mma_drain;
         tc_fence_after();
@@ -231,7 +238,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int kb = 0; kb < p.k_steps; ++kb) {
         // warp-uniform outcome: tcgen05.st below needs all 32 lanes
         if (!__all_sync(0xFFFFFFFFu,
-                        mbar_wait(&full[stage], phase, abort_flag, p.watchdog, WD_STAGING)))
+                        mbar_wait(&sf_loaded[stage], phase, abort_flag, p.watchdog, WD_STAGING)))
           goto staging_done;
         {
           const uint32_t sfa_s = smem_u32(sSFA + stage * SFA_STAGE) + lane * 16;
@@ -287,20 +294,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const int row = mt * BM + quarter * 32 + lane;
       const bool row_ok = row < p.M;
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL + c * 32;
-        FP4_TMEM_LD_32x32b_X32(taddr, r);
-        tmem_ld_wait();
-        if (c == BN / 32 - 1) {
-          // accumulator fully read: let the next tile's MMAs start
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL;
+      if (!OUT_F32) {
+        // bf16: the whole 256-column row fits in 128 registers once packed,
+        // so the accumulator is released before any global store is issued
+        uint32_t packed[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float lo = __fmul_rn(alpha, __uint_as_float(r[2 * j]));
+            const float hi = __fmul_rn(alpha, __uint_as_float(r[2 * j + 1]));
+            __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+            packed[16 * c + j] = *reinterpret_cast<uint32_t*>(&h);
+          }
         }
-        const int n0 = nt * BN + c * 32;
-        if (!row_ok || n0 >= p.N) continue;
-        if (OUT_F32) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        if (row_ok) {
+          uint16_t* out = static_cast<uint16_t*>(p.C) + static_cast<long long>(row) * p.ldc;
+#pragma unroll
+          for (int v = 0; v < BN / 8; ++v) {
+            const int n = nt * BN + 8 * v;
+            if (n < p.N)
+              *reinterpret_cast<uint4*>(out + n) = make_uint4(packed[4 * v], packed[4 * v + 1],
+                                                              packed[4 * v + 2], packed[4 * v + 3]);
+          }
+        }
+      } else {
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
+          tmem_ld_wait();
+          if (c == BN / 32 - 1) {
+            // accumulator fully read: let the next tile's MMAs start
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          const int n0 = nt * BN + c * 32;
+          if (!row_ok || n0 >= p.N) continue;
           float* out = static_cast<float*>(p.C) + static_cast<long long>(row) * p.ldc + n0;
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
@@ -311,22 +348,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               o.z = __fmul_rn(alpha, __uint_as_float(r[4 * v + 2]));
               o.w = __fmul_rn(alpha, __uint_as_float(r[4 * v + 3]));
               *reinterpret_cast<float4*>(out + 4 * v) = o;
-            }
-          }
-        } else {
-          uint16_t* out = static_cast<uint16_t*>(p.C) + static_cast<long long>(row) * p.ldc + n0;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            if (n0 + 8 * v < p.N) {
-              uint32_t w[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float lo = __fmul_rn(alpha, __uint_as_float(r[8 * v + 2 * j]));
-                const float hi = __fmul_rn(alpha, __uint_as_float(r[8 * v + 2 * j + 1]));
-                __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-                w[j] = *reinterpret_cast<uint32_t*>(&h);
-              }
-              *reinterpret_cast<uint4*>(out + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
         }
