@@ -97,3 +97,43 @@ def test_prefill_full_size_sampled(ops, orc, M, N, K, fmt, dt):
     c_ref = orc.gemm(orc.dequant(ca, sa, fmt, ga), orc.dequant(cw, sw, fmt, gw))
     ok, worst, where = gemm_close(c[rt.cuda()][:, ct.cuda()], c_ref, DT[dt])
     assert ok, f"worst err/bound {worst:.3g} at {where}"
+
+
+FUSED_RAGGED = [(1, 8, 32), (5, 264, 2880), (16, 520, 1056), (17, 136, 96), (32, 1024, 4096),
+                (32, 14336, 256), (3, 4096, 8192)]
+
+
+@pytest.mark.parametrize("M,N,K", FUSED_RAGGED)
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_fused_ragged_shapes(ops, orc, M, N, K, fmt, dt):
+    """Split-K and single-slice grids, padded activation rows, K tails."""
+    a = inputs.random_bf16(300 + M, (M, K))
+    w = inputs.random_bf16(400 + N, (N, K), 0.02)
+    run_pair(ops, orc, a, w, fmt, dt, fused=True)
+
+
+@pytest.mark.parametrize("g", [1.0, 0.01])
+def test_fused_static_global_scale(ops, orc, g):
+    M, N, K = 8, 512, 2048
+    a = inputs.random_bf16(500, (M, K))
+    w = inputs.random_bf16(501, (N, K), 0.02)
+    ca, sa, ga = orc.quantize(a, 0, g)
+    wq_ref = orc.quantize(w, 0)
+    c_ref = orc.gemm(orc.dequant(ca, sa, 0, ga), orc.dequant(*wq_ref[:2], 0, wq_ref[2]))
+    wq = ops.quantize_weights(w.cuda(), 0)
+    c = ops.gemm_fused(a.cuda(), wq, torch.float32,
+                       g_a=torch.tensor([g], dtype=torch.float32, device="cuda"))
+    torch.cuda.synchronize()
+    ok, worst, where = gemm_close(c, c_ref, torch.float32)
+    assert ok, f"worst err/bound {worst:.3g} at {where}"
+
+
+def test_fused_repeated_calls_are_deterministic(ops):
+    """The split-K reduction runs in slice order: repeated calls give identical bits."""
+    a, w = inputs.decode(32, 4096, 14336)
+    wq = ops.quantize_weights(w.cuda(), 0)
+    x = a.cuda()
+    outs = [ops.gemm_fused(x, wq, torch.float32).clone() for _ in range(3)]
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
