@@ -125,6 +125,149 @@ def cpu_baseline(sample_rows=256, sample_cols=4096, seconds_target=10.0):
     return flop / t_total / 1e12, oracle.threads(), desc
 
 
+DECODE_SHAPES = [(M, N, K) for (N, K) in ((4096, 4096), (14336, 4096), (4096, 14336))
+                 for M in (1, 8, 32)]
+SWEEP_SHAPES = [(M, K) for M in (1, 32, 512, 8192) for K in (2880, 8192, 16384)]
+L2_BYTES = 126 * 2 ** 20
+
+
+def flush_l2(torch, buf_w, buf_r):
+    """Evict L2: write a buffer twice its size, then read another one, so the
+    timed kernel meets clean (not dirty) lines."""
+    buf_w.zero_()
+    buf_r.sum()
+
+
+def decode_bytes(M, N, K):
+    """Algorithmic bytes of one fused decode call: packed weights + their
+    E4M3 scales, the bf16 activation read once, the bf16 output written."""
+    return N * K * 0.5625 + M * K * 2 + M * N * 2
+
+
+def measure_decode(torch, ops, L, inputs, dev, hbm_peak, shapes=None):
+    """fp4_gemm_fused on the decode shapes: (i) one call after an L2 flush,
+    (ii) back-to-back calls inside one captured CUDA graph, cycling through
+    enough weight copies that every call streams its weights from HBM."""
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    out = []
+    w_cache = {}
+    for (M, N, K) in (shapes or DECODE_SHAPES):
+        if (N, K) not in w_cache:
+            w_cache.clear()
+            _, w = inputs.decode(1, N, K)
+            w_cache[(N, K)] = ops.quantize_weights(w.to(dev), L.FP4_NVFP4)
+        wq0 = w_cache[(N, K)]
+        x = inputs.random_bf16(7, (M, K)).to(dev)
+        wbytes = wq0.codes.numel() + wq0.scales.numel()
+        copies = max(2, -(-3 * L2_BYTES // wbytes))
+        wqs = [ops.Quantized(wq0.codes.clone(), wq0.scales.clone(), wq0.g.clone(), wq0.fmt,
+                             wq0.layout, wq0.rows, wq0.K) for _ in range(copies)]
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        g_out = torch.empty(1, dtype=torch.float32, device=dev)
+        for wq in wqs[:2]:
+            ops.gemm_fused(x, wq, out=c, g_out=g_out)
+        torch.cuda.synchronize(dev)
+        # (i) single call, cold L2
+        cold = []
+        for i in range(5):
+            flush_l2(torch, flush, flush_r)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ops.gemm_fused(x, wqs[i % copies], out=c, g_out=g_out)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            cold.append(e0.elapsed_time(e1) * 1e3)
+        # (ii) graph of `copies` back-to-back calls
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for wq in wqs:
+                ops.gemm_fused(x, wq, out=c, g_out=g_out)
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        reps = max(3, int(2000 // copies))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+        gbs = decode_bytes(M, N, K) / (us * 1e-6) / 1e9
+        out.append({"M": M, "N": N, "K": K, "us_graph": round(us, 3),
+                    "gbs_graph": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 4),
+                    "us_cold_single": round(float(np.median(cold)), 3),
+                    "weight_copies": copies})
+        del graph, wqs
+    return out
+
+
+def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak):
+    """fp4_quantize_act on the activation-quantize sweep, L2 flushed before
+    every call.  Reports GB/s with single-pass bytes (2.5625 B/elem NVFP4,
+    2.53125 MXFP4) and, for the DYNAMIC NVFP4 run, with both reads of the
+    amax pass (4.5625 B/elem)."""
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    sp = torch.cuda.current_stream(dev).cuda_stream
+    res = []
+    for (M, K) in SWEEP_SHAPES:
+        x = inputs.act_sweep(M, K).to(dev)
+        for fmt, gmode, name in ((0, 0, "nvfp4_dynamic"), (0, 1, "nvfp4_static"), (1, 0, "mxfp4")):
+            codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+            scales = torch.empty(L.fp4_scale_bytes(M, K, fmt, 0), dtype=torch.uint8, device=dev)
+            g = torch.full((1,), 0.05, dtype=torch.float32, device=dev)
+            wsb = L.fp4_workspace_bytes(M, 0, K, fmt)
+            ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+            ts = []
+            for i in range(8):
+                flush_l2(torch, flush, flush_r)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                st = L.fp4_quantize_act(x.data_ptr(), M, K, fmt, 0, gmode, g.data_ptr(),
+                                        codes.data_ptr(), scales.data_ptr(), ws.data_ptr(), wsb, sp)
+                e1.record()
+                torch.cuda.synchronize(dev)
+                assert st == 0
+                if i >= 3:
+                    ts.append(e0.elapsed_time(e1) * 1e3)
+            us = float(np.median(ts))
+            single = (2.5625 if fmt == 0 else 2.53125) * M * K
+            row = {"M": M, "K": K, "variant": name, "us": round(us, 3),
+                   "gbs_single_pass": round(single / (us * 1e-6) / 1e9, 1)}
+            if gmode == 0 and fmt == 0:
+                two = 4.5625 * M * K
+                row["gbs_two_reads"] = round(two / (us * 1e-6) / 1e9, 1)
+                row["frac_hbm_two_reads"] = round(two / (us * 1e-6) / 1e9 / hbm_peak, 4)
+            row["frac_hbm_single_pass"] = round(single / (us * 1e-6) / 1e9 / hbm_peak, 4)
+            res.append(row)
+    return res
+
+
+def run_part(args, rank):
+    """One supplementary measurement alone (profiling aid)."""
+    import torch
+    from mxfp4_block_scaled_fp4_b200 import fp4lib as L, inputs, ops
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    L.lib()
+    peaks, _ = load_peaks()
+    line = {"metric": METRIC, "impl": "ours", "part": args.only}
+    if args.only == "decode":
+        shapes = None
+        if args.decode_shape:
+            shapes = [tuple(int(v) for v in args.decode_shape.split(","))]
+        line["decode"] = measure_decode(torch, ops, L, inputs, dev, peaks["hbm_gbs"], shapes)
+    else:
+        line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args, rank):
     if rank != 0:
         return 0
@@ -150,6 +293,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-suite", action="store_true",
+                    help="skip the decode and quantize-sweep measurements")
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quantize"],
+                    help="run one part only (profiling); the JSON line then carries that part")
+    ap.add_argument("--decode-shape", default=None, help="M,N,K: restrict the decode part")
     ap.add_argument("--shape", default=None,
                     help="M,N,K override (profiling of smaller cases); default 8192,28672,8192")
     args = ap.parse_args()
@@ -164,6 +312,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.only in ("decode", "quantize"):
+        return run_part(args, rank)
     if args.warmup < 3:
         args.warmup = 3
 
@@ -307,6 +457,11 @@ def main():
         "e2e": {"value": FLOP * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": a_host.numel() * 2, "d2h_bytes_per_step": c_host.numel() * 2},
     }
+    if not args.no_suite:
+        line["decode"] = measure_decode(torch, ops, L, inputs, dev, peaks["hbm_gbs"])
+        line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"])
+        line["gpu_launches_note"] = ("gpu_launches counts the timed prefill steps only; the "
+                                     "decode and sweep objects are timed separately")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         val, cores, desc = cpu_baseline()
         line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores,

@@ -133,14 +133,19 @@ fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const flo
                       void* ws, size_t ws_bytes, void* stream);
 
 /* Small-M path (decode): quantize the bf16 activation a [M, K] on the fly
- * and multiply it with pre-quantized weights in one launch sequence, without
- * a round trip of the quantized activation through global memory.
+ * and multiply it with pre-quantized weights, as one chain of programmatic
+ * dependent launches on `stream`: amax (DYNAMIC only) -> quantize (into the
+ * workspace) -> a swap-AB, split-K tcgen05 GEMM for M <= 32 that starts
+ * streaming the weights before the quantized activation is ready.
  * "FP4 n'existe pas", runtime survey (quantization, scaling, matmul and
- * de-scaling fused in one launch); the small-M regime: "Hardware FP4
+ * de-scaling chained in one go); the small-M regime: "Hardware FP4
  * inference for speech on Blackwell", section "Do the FP4 tensor cores even
  * engage?".  g_a: DYNAMIC writes it, STATIC reads it (NVFP4; MXFP4 ignores
  * it).  Results equal fp4_quantize_act followed by fp4_gemm up to FP32
- * summation order.  Requires M <= 32 (FP4_ERR_UNSUPPORTED_SHAPE otherwise). */
+ * summation order; the split-K reduction runs in a fixed order, so repeated
+ * calls give identical bits.  Requires 1 <= M <= 32 (M == 0 is a no-op;
+ * FP4_ERR_UNSUPPORTED_SHAPE above 32).  The workspace (fp4_workspace_bytes)
+ * holds the partial maxima and the quantized activation. */
 fp4_status_t fp4_gemm_fused(const void* a, const uint8_t* w_codes, const uint8_t* w_scales,
                             const float* g_w, int M, int N, int K, fp4_format_t fmt,
                             fp4_global_mode_t gmode, float* g_a,

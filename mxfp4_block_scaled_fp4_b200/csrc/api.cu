@@ -182,6 +182,7 @@ fp4_status_t fp4_gemm_fused(const void* x, const uint8_t* w_codes, const uint8_t
   if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (N % 8 != 0 || M > 32) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (M == 0 || N == 0) return FP4_OK;   // nothing is read or written
+  if (!fp4::fused_supported(M, N, K)) return FP4_ERR_UNSUPPORTED_SHAPE;
   const bool nv = fmt == FP4_NVFP4;
   if (!x || !w_codes || !w_scales || !C || !ws || (nv && (!g_a || !g_w)))
     return FP4_ERR_INVALID_ARG;

@@ -7,31 +7,36 @@
 // tensor cores even engage?".  Same arithmetic as fp4_quantize_act followed
 // by fp4_gemm (bit-identical codes and scales), up to FP32 summation order.
 //
-// Two launches per call:
-//  prologue  (tiny) zeroes the split-K arrival counters and, for a DYNAMIC
-//            global scale, writes one partial amax per CTA.  It lets the
-//            main kernel launch right away (programmatic dependent launch),
-//            so weight streaming starts while the amax is still running.
+// One or two launches per call:
+//  prologue  (DYNAMIC global scale only) one partial amax per CTA.  Every
+//            launch is a programmatic dependent of the one before it, and
+//            every kernel here releases its dependent early, so a kernel's
+//            weight streaming starts while its predecessor still runs; a
+//            kernel reads the activation only after griddepcontrol.wait.
 //  main      swap-AB: the weights are the 128-row "A" operand of
 //            tcgen05.mma kind::mxf4nvf4 and the <= 32 activation rows are the
 //            16- or 32-wide "B" operand.  Grid = N/128 weight tiles x S
-//            split-K slices.  Per CTA:
+//            split-K slices, S chosen so the grid fits one wave.  Per CTA:
 //     warp 0     TMA: weight tiles (16 KiB per 256 K) + their scale atoms
 //                through a 4-stage ring;
 //     warp 1     MMA issuer;
-//     warps 2-5  (a) after griddepcontrol.wait: global scale, then quantize
-//                    the CTA's K slice of the activation into shared memory
-//                    (128-byte swizzled K-major rows, the MMA's B layout) and
-//                    its scales into tensor memory (tcgen05.st);
-//                (b) stage each ring stage's weight scales into tensor
-//                    memory; (c) epilogue: accumulator -> C (S = 1) or ->
-//                    split-K partials; the last CTA of a tile sums the S
-//                    partials in slice order (deterministic) and writes C.
+//     warps 2-5  after griddepcontrol.wait: global scale; then per 256-K
+//                step, quantize the activation rows into shared memory
+//                (128-byte swizzled K-major rows, the MMA's B layout) and
+//                their scales into tensor memory (tcgen05.st), loads of
+//                the next step in flight meanwhile; finally the epilogue.
+//     Weight scales go to tensor memory with tcgen05.cp from the MMA
+//     thread: at decode sizes the tensor pipe has slack for it.
+//  With S > 1 slices the S CTAs of a weight tile form a thread-block
+//  cluster: each leaves its FP32 partial in shared memory and CTA s sums
+//  rows m = s, s + S, ... over the S partials in slice order through
+//  distributed shared memory (deterministic, no global round trip).
 #include <cuda_bf16.h>
 
 #include <algorithm>
 
 #include "internal.h"
+#include "codec.cuh"
 #include "ptx.cuh"
 
 namespace fp4 {
@@ -43,46 +48,65 @@ constexpr int FBK = 256;                 // K per ring stage
 constexpr int FBK_BYTES = FBK / 2;
 constexpr int FSTAGES = 4;
 constexpr int FW_STAGE = FBM * FBK_BYTES;   // 16 KiB
-constexpr int FSF_STAGE = 4 * 512;          // up to 4 scale atoms
-constexpr int kMaxStepsPerSplit = 16;       // K slice <= 4096 per CTA
+constexpr int FSF_STAGE = 4 * 512;          // up to 4 weight-scale atoms
+constexpr int kMaxSplits = 8;               // portable cluster size
+constexpr int kMaxStepsPerSplit = 26;       // activation scales of a slice fit tensor memory
 constexpr int kFusedThreads = 192;          // TMA, MMA, 4 worker warps
-constexpr int kTargetCtas = 148;            // one CTA per B200 SM
+constexpr int kTargetCtas = 148;            // SMs of a B200
+constexpr int kSmemPerSm = 227 * 1024;      // shared memory a B200 SM offers to CTAs
+constexpr int kStageBudget = 64 * 1024;     // bf16 activation staging (two buffers)
 constexpr int kPrologueThreads = 256;
 constexpr int kMaxPrologueCtas = 148;
 // Tensor-memory columns.  Every scale-factor address an MMA gets is a
-// multiple of 4 columns (16 bytes), the alignment the passing GEMM uses: a
-// fault was seen on B200 when activation scales sat at columns 4i + k.
-constexpr uint32_t F_TMEM_COLS = 512;
+// multiple of 4 columns (16 bytes): a misaligned-address fault was seen on
+// B200 when scales sat at columns 4i + k.
 constexpr uint32_t F_ACC_COL = 0;           // <= 32 fp32 columns
 constexpr uint32_t F_SFA_COL = 32;          // weight scales: 16 columns per ring stage
-constexpr uint32_t F_SFB_COL = 128;         // activation scales: 4 columns per scale word
+constexpr uint32_t F_SFB_COL = 96;          // activation scales: 16 columns per K step
+inline int tmem_cols_for(int steps) { return (F_SFB_COL + 16 * steps) <= 256 ? 256 : 512; }
 
 size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
 struct Plan {
   int n_tiles, k_steps, splits, steps_max, nmma_n;
-  size_t ws_partial_off, ws_counter_off, ws_sum_off, ws_bytes;
-  int smem_bytes;
+  int smem_bytes, tmem_cols, group;
+  bool ok;
 };
 
-Plan make_plan(int M, int N, int K, int fmt) {
+// Steps of bf16 activation staged per group (double-buffered cp.async).
+int group_steps(int M, int steps) {
+  const int per_step = M * FBK * 2;                 // bf16 bytes of one 256-K step
+  return std::max(1, std::min(steps, kStageBudget / (2 * per_step)));
+}
+
+int plan_smem(int M, int steps, int nmma_n) {
+  const int gs = group_steps(M, steps);
+  return 1024 + FSTAGES * (FW_STAGE + FSF_STAGE) + steps * nmma_n * FBK_BYTES +
+         steps * nmma_n * 16 + 2 * gs * M * FBK * 2 + 256;
+}
+
+// Split count: the largest S <= 8 whose whole grid (N/128 tiles x S) fits in
+// one wave, counting two CTAs per SM when shared and tensor memory allow.
+Plan make_plan(int M, int N, int K) {
   Plan p{};
   p.n_tiles = (N + FBM - 1) / FBM;
   p.k_steps = (K + FBK - 1) / FBK;
-  int s = (kTargetCtas + p.n_tiles - 1) / p.n_tiles;
-  s = std::max(s, (p.k_steps + kMaxStepsPerSplit - 1) / kMaxStepsPerSplit);
-  p.splits = std::max(1, std::min(s, p.k_steps));
-  p.steps_max = (p.k_steps + p.splits - 1) / p.splits;
   p.nmma_n = M <= 16 ? 16 : 32;
-  p.ws_partial_off = 0;
-  p.ws_counter_off = align256(static_cast<size_t>(kMaxPrologueCtas) * sizeof(unsigned));
-  p.ws_sum_off = p.ws_counter_off + align256(static_cast<size_t>(p.n_tiles) * sizeof(unsigned));
-  const size_t sums = p.splits > 1 ? static_cast<size_t>(p.n_tiles) * p.splits * M * FBM * 4 : 0;
-  p.ws_bytes = p.ws_sum_off + align256(sums);
-  const int act_bytes = p.steps_max * p.nmma_n * FBK_BYTES;
-  const int sf_scratch = p.nmma_n * p.steps_max * 16;
-  p.smem_bytes = 1024 + FSTAGES * (FW_STAGE + FSF_STAGE) + act_bytes + sf_scratch + 256;
-  (void)fmt;
+  int best = 0;
+  for (int s = 1; s <= kMaxSplits && s <= p.k_steps; ++s) {
+    const int steps = (p.k_steps + s - 1) / s;
+    if (steps > kMaxStepsPerSplit) continue;
+    const int smem = plan_smem(M, steps, p.nmma_n);
+    if (smem > kSmemPerSm) continue;
+    const int per_sm = (smem <= kSmemPerSm / 2 && tmem_cols_for(steps) <= 256) ? 2 : 1;
+    if (best == 0 || p.n_tiles * s <= kTargetCtas * per_sm) best = s;
+  }
+  p.ok = best > 0;
+  p.splits = best > 0 ? best : 1;
+  p.steps_max = (p.k_steps + p.splits - 1) / p.splits;
+  p.group = group_steps(M, p.steps_max);
+  p.smem_bytes = plan_smem(M, p.steps_max, p.nmma_n);
+  p.tmem_cols = tmem_cols_for(p.steps_max);
   return p;
 }
 
@@ -92,13 +116,11 @@ struct FParams {
   const float* g_w;
   float* g_a;
   const unsigned* amax_partial;
-  unsigned* counters;
-  float* sums;
   void* C;
   long long ldc;
   int M, N, K;
   int dynamic, out_f32;
-  int n_tiles, k_steps, splits, steps_max, nmma_n, ncb, n_partial;
+  int n_tiles, k_steps, splits, steps_max, nmma_n, ncb, n_partial, tmem_cols, group;
   unsigned* watchdog;
 };
 
@@ -112,6 +134,28 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void workers_sync() {   // named barrier of the 4 worker warps
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_peer_f32(uint32_t local_saddr, uint32_t rank) {
+  uint32_t remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// 16-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+               ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ uint4 ld_nc16(const void* p) {
   uint4 v;
@@ -120,68 +164,28 @@ __device__ __forceinline__ uint4 ld_nc16(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ unsigned mag_max8(uint4 v) {
-  unsigned m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                        __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-  return m;
-}
-
-// ---- element codecs (same rounding steps as the stand-alone quantizer)
-__device__ __forceinline__ unsigned f_to_e4m3(float v) {
-  unsigned short r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
-  return r & 0xFFu;
-}
-__device__ __forceinline__ float f_e4m3_value(unsigned c) {
-  const unsigned e = c >> 3, m = c & 7u;
-  if (e == 0) return __uint2float_rn(m) * 0.001953125f;
-  return __uint_as_float(((e + 120u) << 23) | (m << 20));
-}
-__device__ __forceinline__ unsigned f_e2m1x8(float v0, float v1, float v2, float v3, float v4,
-                                             float v5, float v6, float v7) {
-  unsigned out;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(out)
-      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
-  return out;
-}
-__device__ __forceinline__ unsigned f_quant8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
-                                             float r) {
-  auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
-  auto hi = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
-  auto sg = [](uint32_t w) { return ((w >> 12) & 0x8u) | ((w >> 24) & 0x80u); };
-  const unsigned q = f_e2m1x8(__fmul_rn(lo(w0), r), __fmul_rn(hi(w0), r), __fmul_rn(lo(w1), r),
-                              __fmul_rn(hi(w1), r), __fmul_rn(lo(w2), r), __fmul_rn(hi(w2), r),
-                              __fmul_rn(lo(w3), r), __fmul_rn(hi(w3), r));
-  return q | sg(w0) | sg(w1) << 8 | sg(w2) << 16 | sg(w3) << 24;
-}
-__device__ __forceinline__ int f_floor_log2(float b) {
-  const unsigned u = __float_as_uint(b);
-  const int ex = static_cast<int>((u >> 23) & 0xFFu);
-  if (ex != 0) return ex - 127;
-  return (31 - __clz(u & 0x7FFFFFu)) - 149;
+__device__ __forceinline__ void store_out(const FParams& p, int m, int n, float c) {
+  if (p.out_f32)
+    static_cast<float*>(p.C)[m * p.ldc + n] = c;
+  else
+    static_cast<__nv_bfloat16*>(p.C)[m * p.ldc + n] = __float2bfloat16_rn(c);
 }
 
 // ------------------------------------------------------------ prologue
 
+// DYNAMIC global scale: one partial amax per CTA.  Launched as a
+// programmatic dependent of the previous kernel, it lets the main kernel
+// launch at once, so the weights start streaming while this runs.
 __global__ void __launch_bounds__(kPrologueThreads)
-    fused_prologue_kernel(const uint4* __restrict__ a, long long n_vec, int dynamic,
-                          unsigned* __restrict__ partial, unsigned* __restrict__ counters,
-                          int n_counters) {
-  grid_dep_launch();   // the main kernel may start streaming weights now
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_counters; i += gridDim.x * blockDim.x)
-    counters[i] = 0;
-  if (!dynamic) return;
+    fused_amax_kernel(const uint4* __restrict__ a, long long n_vec,
+                      unsigned* __restrict__ partial) {
+  grid_dep_launch();   // the main kernel may launch and prefetch weights
+  grid_dep_wait();     // the kernel that wrote `a` (if any) has finished
   unsigned m = 0;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_vec;
        i += static_cast<long long>(gridDim.x) * blockDim.x)
     m = __vmaxu2(m, mag_max8(ld_nc16(a + i)));
-  m = max(m & 0xFFFFu, m >> 16);
+  m = fold_u16x2(m);
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   __shared__ unsigned red[kPrologueThreads / 32];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -205,19 +209,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   uint8_t* sSF = sW + FSTAGES * FW_STAGE;
   uint8_t* sAct = sSF + FSTAGES * FSF_STAGE;                 // 1024-aligned
   const int act_chunk = p.nmma_n * FBK_BYTES;                 // bytes per 256 K
-  uint8_t* sScr = sAct + p.steps_max * act_chunk;             // activation scale bytes
-  const int scr_row = p.steps_max * 16;                       // scale bytes per row
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sScr + p.nmma_n * scr_row);
+  uint8_t* sScr = sAct + p.steps_max * act_chunk;             // per step: nmma_n x 16 scale bytes
+  const int scr_step = p.nmma_n * 16;
+  uint8_t* sX = sScr + p.steps_max * scr_step;                // bf16 staging, two group buffers
+  const int x_row = p.group * FBK * 2;                        // bytes of one row in a buffer
+  const int x_buf = p.M * x_row;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sX + 2 * x_buf);
   uint64_t* full = bars;
   uint64_t* empty = full + FSTAGES;
   uint64_t* sf_loaded = empty + FSTAGES;
   uint64_t* sf_full = sf_loaded + FSTAGES;
-  uint64_t* act_ready = sf_full + FSTAGES;
-  uint64_t* acc_full = act_ready + 1;
+  uint64_t* acc_full = sf_full + FSTAGES;
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x / p.splits, split = blockIdx.x % p.splits;
@@ -233,31 +238,40 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       mbar_init(&sf_loaded[s], 1);
       mbar_init(&sf_full[s], 4);
     }
-    mbar_init(act_ready, 4);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
-    *last_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm_w);
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, F_TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  // every CTA of this grid is resident: the next kernel in the stream may
+  // launch now and start streaming its own weights into free SM resources
+  grid_dep_launch();
+  // tensor memory is allocated by warp 1 while warp 0 already streams
+  // weights; warps 1-5 meet on named barrier 2 before using it
+  uint32_t tmem = 0;
+  if (warp >= 1) {
+    if (warp == 1) {
+      tmem_alloc(tmem_slot, static_cast<uint32_t>(p.tmem_cols));
+      tmem_relinquish();
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 2, 160;" ::: "memory");
+    tc_fence_after();
+    tmem = *tmem_slot;
+  }
+  bool epilogue_ok = false;   // workers: the accumulator was read
+  float alpha = 1.0f;         // workers: g_a * g_w (NVFP4) or 1
 
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------ TMA producer
-    uint32_t armed = 0, armed_parity = 0;
-    for (int i = 0; i < n_steps; ++i) {
-      const int stage = i % FSTAGES;
-      const uint32_t phase = static_cast<uint32_t>(i / FSTAGES) & 1u;
-      if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.watchdog, WD_PRODUCER)) goto p_drain;
-      {
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      uint32_t armed = 0, armed_parity = 0;
+      for (int i = 0; i < n_steps; ++i) {
+        const int stage = i % FSTAGES;
+        const uint32_t phase = static_cast<uint32_t>(i / FSTAGES) & 1u;
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.watchdog, WD_PRODUCER)) break;
         const int ks = s_lo + i;
         const int cb0 = ks * kAtoms;
         const int atoms = min(kAtoms, p.ncb - cb0);
@@ -270,60 +284,63 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
       }
-    }
-    goto p_done;
-  p_drain:
-    for (int s = 0; s < FSTAGES; ++s)
-      if (armed & (1u << s)) {
-        mbar_wait_drain(&sf_loaded[s], (armed_parity >> s) & 1u, p.watchdog);
-        mbar_wait_drain(&full[s], (armed_parity >> s) & 1u, p.watchdog);
+      if (*abort_flag) {
+        for (int s = 0; s < FSTAGES; ++s)
+          if (armed & (1u << s)) {
+            mbar_wait_drain(&sf_loaded[s], (armed_parity >> s) & 1u, p.watchdog);
+            mbar_wait_drain(&full[s], (armed_parity >> s) & 1u, p.watchdog);
+          }
       }
-  p_done:;
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------- MMA issuer
-    if (!mbar_wait(act_ready, 0, abort_flag, p.watchdog, WD_MMA_FULL)) goto m_drain;
-    tc_fence_after();
-    for (int i = 0; i < n_steps; ++i) {
-      const int stage = i % FSTAGES;
-      const uint32_t phase = static_cast<uint32_t>(i / FSTAGES) & 1u;
-      if (!mbar_wait(&full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) goto m_drain;
-      if (!mbar_wait(&sf_full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) goto m_drain;
-      tc_fence_after();
-      {
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      bool ok = true;
+      for (int i = 0; i < n_steps && ok; ++i) {
+        const int stage = i % FSTAGES;
+        const uint32_t phase = static_cast<uint32_t>(i / FSTAGES) & 1u;
+        // sf_full[stage]: the workers wrote this step's activation (codes and
+        // scales) and the stage's weight scales
+        ok = mbar_wait(&full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL) &&
+             mbar_wait(&sf_full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL);
+        if (!ok) break;
+        tc_fence_after();
         const int kglob = (s_lo + i) * FBK;
         const int n_mma = min(4, (p.K - kglob + 63) / 64);
         const uint32_t w_s = smem_u32(sW + stage * FW_STAGE);
         const uint32_t x_s = smem_u32(sAct + i * act_chunk);
         const uint32_t sfa = tmem + F_SFA_COL + stage * 16;
+        const uint32_t sfb = tmem + F_SFB_COL + i * 16;
         for (int k = 0; k < n_mma; ++k) {
           const uint64_t ad = smem_desc(w_s + k * 32, 16, 1024, kLayoutSwizzle128B);
           const uint64_t bd = smem_desc(x_s + k * 32, 16, 1024, kLayoutSwizzle128B);
           const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
           if (FMT == 0) {
             tc_mma_nvf4(tmem + F_ACC_COL, ad, bd, idesc_fp4(FBM, p.nmma_n, false, 0, 0),
-                        sfa + 4 * k, tmem + F_SFB_COL + 4 * (4 * i + k), acc);
+                        sfa + 4 * k, sfb + 4 * k, acc);
           } else {
             const uint32_t id = 2u * (k & 1);
             tc_mma_mxf4(tmem + F_ACC_COL, ad, bd, idesc_fp4(FBM, p.nmma_n, true, id, id),
-                        sfa + 4 * (k >> 1), tmem + F_SFB_COL + 4 * (2 * i + (k >> 1)), acc);
+                        sfa + 4 * (k >> 1), sfb + 4 * (k >> 1), acc);
           }
         }
+        tc_commit(&empty[stage]);
       }
-      tc_commit(&empty[stage]);
+      if (ok) {
+        tc_commit(acc_full);
+      } else {
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0, p.watchdog);
+      }
     }
-    tc_commit(acc_full);
-    goto m_done;
-  m_drain:
-    tc_commit(drain);
-    mbar_wait_drain(drain, 0, p.watchdog);
-  m_done:;
-  } else if (warp >= 2) {
+    __syncwarp();
+  } else {
     // ------------------------------------------------------------ workers
     const int quarter = warp & 3;
     const int wt = threadIdx.x - 64;                 // 0..127
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    grid_dep_wait();                                 // prologue finished and visible
-    // (a) global scale
+    grid_dep_wait();                                 // amax prologue finished and visible
     float g = 1.0f;
     if (FMT == 0) {
       if (p.dynamic) {
@@ -342,119 +359,172 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       }
     }
     const float six_g = __fmul_rn(6.0f, g);
-    // (a) quantize rows [0, nmma_n) x K slice into the MMA's B layout
-    const int units_per_row = n_steps * 16;
-    const int total = p.nmma_n * units_per_row;      // a multiple of 256
-    for (int u = wt; u < total; u += 128) {
-      const int m = u / units_per_row;
-      const int ku = u - m * units_per_row;
-      const int kg = s_lo * FBK + ku * 16;
-      const bool live = m < p.M && kg < p.K;
-      uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
-      if (live) {
-        const uint16_t* src = p.a + static_cast<long long>(m) * p.K + kg;
-        x0 = ld_nc16(src);
-        x1 = ld_nc16(src + 8);
+    // The activation slice (rows < M, K range of this split) is staged in
+    // groups of p.group steps: cp.async brings group g+1 while group g is
+    // quantized from shared memory into the MMA's B layout (codes) and the
+    // scale scratch; the group's scales then go to tensor memory.  Per step
+    // the workers also move the stage's weight scales into tensor memory and
+    // then signal the MMA thread.  Every worker warp runs every iteration
+    // and every named barrier (an abort skips work, never a barrier).
+    const int k0 = s_lo * FBK;
+    const int chunks_per_row = p.group * FBK / 8;     // 16-byte pieces per row and group
+    auto stage_group = [&](int grp) {
+      const uint32_t dst0 = smem_u32(sX + (grp & 1) * x_buf);
+      const int total = p.M * chunks_per_row;
+      for (int c = wt; c < total; c += 128) {
+        const int m = c / chunks_per_row;
+        const int kk = (c - m * chunks_per_row) * 8 + grp * p.group * FBK;   // within the slice
+        const int kg = k0 + kk;
+        const bool in = kk < n_steps * FBK && kg < p.K;
+        const uint16_t* src = p.a + (in ? static_cast<long long>(m) * p.K + kg : 0);
+        cp_async16(dst0 + m * x_row + (kk - grp * p.group * FBK) * 2, src, in ? 16u : 0u);
       }
-      unsigned mm = __vmaxu2(mag_max8(x0), mag_max8(x1));
-      mm = max(mm & 0xFFFFu, mm >> 16);
-      unsigned sbyte;
-      uint2 q;
-      if (FMT == 0) {
-        sbyte = f_to_e4m3(__fdiv_rn(__uint_as_float(mm << 16), six_g));
-        const float sv = f_e4m3_value(sbyte);
-        if (sv == 0.0f) {
-          q = make_uint2(0, 0);
-        } else {
-          const float r = __frcp_rn(__fmul_rn(sv, g));
-          q = make_uint2(f_quant8(x0.x, x0.y, x0.z, x0.w, r), f_quant8(x1.x, x1.y, x1.z, x1.w, r));
-        }
-      } else {
-        mm = max(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, 1));   // 32-value block = lane pair
-        const float b = __uint_as_float(mm << 16);
-        int e = (b == 0.0f) ? -127 : f_floor_log2(b) - 2;
-        e = max(-127, min(127, e));
-        sbyte = static_cast<unsigned>(e + 127);
-        const float r = __uint_as_float(static_cast<unsigned>(127 - e) << 23);
-        q = make_uint2(f_quant8(x0.x, x0.y, x0.z, x0.w, r), f_quant8(x1.x, x1.y, x1.z, x1.w, r));
-        if (!live) sbyte = 0;
-      }
-      // codes: chunk ku/16, byte (ku%16)*8 of the row, 128-byte swizzle
-      const int chunk = ku >> 4, kb = (ku & 15) * 8;
-      const int off = chunk * act_chunk + (m >> 3) * 1024 + (m & 7) * 128 +
-                      ((((kb >> 4) ^ (m & 7)) << 4) | (kb & 15));
-      *reinterpret_cast<uint2*>(sAct + off) = q;
-      if (FMT == 0)
-        sScr[m * scr_row + ku] = static_cast<uint8_t>(sbyte);
-      else if ((ku & 1) == 0)
-        sScr[m * scr_row + (ku >> 1)] = static_cast<uint8_t>(sbyte);
-    }
-    fence_proxy_async_smem();    // generic-proxy writes -> visible to the tensor core
-    workers_sync();
-    {
-      // activation scales -> tensor memory: lane i (every quarter) holds row i;
-      // word c = scale bytes [4c, 4c+4) of the row (one MMA for NVFP4, two for
-      // MXFP4) goes to column F_SFB_COL + 4c; the other 3 columns hold 0
-      const int words = (FMT == 0) ? n_steps * 4 : n_steps * 2;
-      const uint32_t* row = reinterpret_cast<const uint32_t*>(sScr + lane * scr_row);
-      const bool has_row = lane < p.nmma_n;
-      for (int c0 = 0; c0 < words; c0 += 4) {
-        uint32_t v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          v[j] = ((j & 3) == 0 && has_row && c0 + (j >> 2) < words) ? row[c0 + (j >> 2)] : 0u;
-        tmem_st_x16(tmem + lane_off + F_SFB_COL + 4 * c0, v);
-      }
-      tmem_st_wait();
-    }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(act_ready);
-    // (b) weight scales of each ring stage -> tensor memory (every quarter
-    // gets the 32-row x 16-byte block of each atom).  A failed wait only
-    // leaves the loop: the accumulator wait below then fails fast too, and
-    // all four warps decide together whether to run the epilogue.
+      cp_async_commit();
+    };
+    const int n_groups = (n_steps + p.group - 1) / p.group;
+    if (n_groups > 0) stage_group(0);
     for (int i = 0; i < n_steps; ++i) {
       const int stage = i % FSTAGES;
       const uint32_t phase = static_cast<uint32_t>(i / FSTAGES) & 1u;
+      if (i % p.group == 0) {
+        const int grp = i / p.group;
+        if (grp + 1 < n_groups) {
+          stage_group(grp + 1);
+          cp_async_wait<1>();
+        } else {
+          cp_async_wait<0>();
+        }
+        workers_sync();                             // group grp is in shared memory
+        const uint8_t* xb = sX + (grp & 1) * x_buf;
+        const int g_steps = min(p.group, n_steps - i);
+        // Only rows m < M are quantized: padding rows feed only output
+        // columns that are never stored.  Each thread takes 4 independent
+        // 16-value units per batch (loads, then math, then stores) so their
+        // long rounding chains interleave.
+        const int per_step = p.M * 16;
+        const int units = g_steps * per_step;
+        const int padded = (units + 511) / 512 * 512;   // whole warps in every batch
+        for (int base = 0; base < padded; base += 512) {
+          uint4 x0[4], x1[4];
+          int step_of[4], m_of[4], ku_of[4];
+          bool act[4], live[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int u = base + j * 128 + wt;
+            act[j] = u < units;
+            const int uu = act[j] ? u : 0;
+            const int sl = uu / per_step;
+            const int r = uu - sl * per_step;
+            m_of[j] = r >> 4;
+            ku_of[j] = r & 15;
+            step_of[j] = i + sl;
+            const int kg = k0 + step_of[j] * FBK + ku_of[j] * 16;
+            live[j] = act[j] && kg < p.K;
+            x0[j] = x1[j] = make_uint4(0, 0, 0, 0);
+            if (live[j]) {
+              const uint32_t src = smem_u32(xb + m_of[j] * x_row + (sl * FBK + ku_of[j] * 16) * 2);
+              x0[j] = lds128(src);
+              x1[j] = lds128(src + 16);
+            }
+          }
+          uint2 q[4];
+          unsigned sb[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            unsigned mm = fold_u16x2(__vmaxu2(mag_max8(x0[j]), mag_max8(x1[j])));
+            float rr;
+            if (FMT == 0) {
+              sb[j] = nvfp4_scale(mm, g, six_g, &rr);
+              q[j] = (rr == 0.0f) ? make_uint2(0, 0)
+                                  : make_uint2(quant8(x0[j].x, x0[j].y, x0[j].z, x0[j].w, rr),
+                                               quant8(x1[j].x, x1[j].y, x1[j].z, x1[j].w, rr));
+            } else {
+              mm = max(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, 1));   // 32-value block = lane pair
+              sb[j] = mxfp4_scale(mm, &rr);
+              q[j] = make_uint2(quant8(x0[j].x, x0[j].y, x0[j].z, x0[j].w, rr),
+                                quant8(x1[j].x, x1[j].y, x1[j].z, x1[j].w, rr));
+              if (!live[j]) sb[j] = 0;
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (!act[j]) continue;
+            const int m = m_of[j], ku = ku_of[j], step = step_of[j];
+            // codes: byte ku*8 of row m in the step's chunk, 128-byte swizzle
+            const int kb = ku * 8;
+            const int off = step * act_chunk + (m >> 3) * 1024 + (m & 7) * 128 +
+                            ((((kb >> 4) ^ (m & 7)) << 4) | (kb & 15));
+            *reinterpret_cast<uint2*>(sAct + off) = q[j];
+            uint8_t* scr = sScr + step * scr_step;
+            if (FMT == 0)
+              scr[m * 16 + ku] = static_cast<uint8_t>(sb[j]);
+            else if ((ku & 1) == 0)
+              scr[m * 16 + (ku >> 1)] = static_cast<uint8_t>(sb[j]);
+          }
+        }
+        fence_proxy_async_smem();      // generic-proxy writes -> visible to the tensor core
+        workers_sync();
+        // the group's activation scales -> tensor memory: lane i holds row i;
+        // word c of a step's row goes to column 16 step + 4 c (4-aligned)
+        if (!*abort_flag) {
+          for (int sl = 0; sl < g_steps; ++sl) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (lane < p.M)
+              w = *reinterpret_cast<const uint4*>(sScr + (i + sl) * scr_step + lane * 16);
+            uint32_t bw[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) bw[j] = 0u;
+            bw[0] = w.x;
+            bw[4] = w.y;
+            if (FMT == 0) {
+              bw[8] = w.z;
+              bw[12] = w.w;
+            }
+            tmem_st_x16(tmem + lane_off + F_SFB_COL + (i + sl) * 16, bw);
+          }
+        }
+      }
+      // weight scales of this stage -> tensor memory (every quarter gets the
+      // 32-row x 16-byte block of each atom); the wait on sf_loaded also
+      // keeps this arrival within one phase of the MMA thread's wait
       if (!__all_sync(0xFFFFFFFFu,
                       mbar_wait(&sf_loaded[stage], phase, abort_flag, p.watchdog, WD_STAGING)))
-        break;
+        continue;
       {
         const uint32_t src = smem_u32(sSF + stage * FSF_STAGE) + lane * 16;
-        uint32_t v[4 * kAtoms];
+        uint32_t v[16];
 #pragma unroll
         for (int a = 0; a < kAtoms; ++a) {
           const uint4 x = lds128(src + a * 512);
           v[4 * a] = x.x; v[4 * a + 1] = x.y; v[4 * a + 2] = x.z; v[4 * a + 3] = x.w;
         }
-        const uint32_t dst = tmem + lane_off + F_SFA_COL + stage * 16;
-        if (kAtoms == 4) tmem_st_x16(dst, v); else tmem_st_x8(dst, v);
+        if (kAtoms == 4) tmem_st_x16(tmem + lane_off + F_SFA_COL + stage * 16, v);
+        else tmem_st_x8(tmem + lane_off + F_SFA_COL + stage * 16, v);
         tmem_st_wait();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sf_full[stage]);
     }
-    // (c) epilogue
+    // (4) accumulator -> C directly (one slice) or -> this CTA's partial
+    //     in shared memory (several slices: a cluster reduces them below)
     {
-      const bool ok =
+      const bool done =
           __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, abort_flag, p.watchdog, WD_EPILOGUE));
-      workers_sync();               // every worker warp reaches this barrier
-      if (!ok || *abort_flag) goto w_done;
+      workers_sync();
+      epilogue_ok = done && !*abort_flag;
     }
-    tc_fence_after();
-    {
+    if (epilogue_ok) {
+      tc_fence_after();
       uint32_t r[32];
       const uint32_t taddr = tmem + lane_off + F_ACC_COL;
       if (p.nmma_n == 16) {
-        uint32_t* rr = r;
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
             "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-            : "=r"(rr[0]), "=r"(rr[1]), "=r"(rr[2]), "=r"(rr[3]), "=r"(rr[4]), "=r"(rr[5]),
-              "=r"(rr[6]), "=r"(rr[7]), "=r"(rr[8]), "=r"(rr[9]), "=r"(rr[10]), "=r"(rr[11]),
-              "=r"(rr[12]), "=r"(rr[13]), "=r"(rr[14]), "=r"(rr[15])
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+              "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+              "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
             : "r"(taddr));
       } else {
         FP4_TMEM_LD_32x32b_X32(taddr, r);
@@ -462,53 +532,40 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       tmem_ld_wait();
       const int nloc = quarter * 32 + lane;          // weight row within the tile
       const int n = tile * FBM + nloc;
-      const float alpha = (FMT == 0) ? __fmul_rn(g, *p.g_w) : 1.0f;
       if (p.splits == 1) {
+        const float alpha1 = (FMT == 0) ? __fmul_rn(g, *p.g_w) : 1.0f;
         if (n < p.N) {
 #pragma unroll
-          for (int m = 0; m < 32; ++m) {
-            if (m >= p.M) break;
-            const float c = __fmul_rn(alpha, __uint_as_float(r[m]));
-            if (p.out_f32)
-              static_cast<float*>(p.C)[m * p.ldc + n] = c;
-            else
-              static_cast<__nv_bfloat16*>(p.C)[m * p.ldc + n] = __float2bfloat16_rn(c);
-          }
+          for (int m = 0; m < 32; ++m)
+            if (m < p.M) store_out(p, m, n, __fmul_rn(alpha1, __uint_as_float(r[m])));
         }
       } else {
-        float* mine = p.sums + (static_cast<long long>(tile) * p.splits + split) * p.M * FBM;
+        float* part = reinterpret_cast<float*>(sW);  // the ring is idle now
 #pragma unroll
-        for (int m = 0; m < 32; ++m) {
-          if (m >= p.M) break;
-          mine[m * FBM + nloc] = __uint_as_float(r[m]);
-        }
-        __threadfence();
-        workers_sync();
-        if (wt == 0) {
-          const unsigned prev = atomicAdd(&p.counters[tile], 1u);
-          *last_flag = (prev == static_cast<unsigned>(p.splits - 1)) ? 1 : 0;
-        }
-        workers_sync();
-        if (*last_flag) {
-          __threadfence();
-          if (n < p.N) {
-            const float* base = p.sums + static_cast<long long>(tile) * p.splits * p.M * FBM;
-            for (int m = 0; m < p.M; ++m) {
-              float acc = 0.0f;
-              for (int s = 0; s < p.splits; ++s)
-                acc = __fadd_rn(acc, __ldcg(base + (static_cast<long long>(s) * p.M + m) * FBM + nloc));
-              const float c = __fmul_rn(alpha, acc);
-              if (p.out_f32)
-                static_cast<float*>(p.C)[m * p.ldc + n] = c;
-              else
-                static_cast<__nv_bfloat16*>(p.C)[m * p.ldc + n] = __float2bfloat16_rn(c);
-            }
-          }
-          if (wt == 0) p.counters[tile] = 0;
-        }
+        for (int m = 0; m < 32; ++m)
+          if (m < p.M) part[m * FBM + nloc] = __uint_as_float(r[m]);
       }
     }
-  w_done:;
+    alpha = (FMT == 0) ? __fmul_rn(g, *p.g_w) : 1.0f;
+  }
+
+  if (p.splits > 1) {
+    // every CTA of the tile's cluster has written its partial sums
+    cluster_sync_all();
+    if (warp >= 2 && epilogue_ok) {
+      const int wt = threadIdx.x - 64;
+      const int n = tile * FBM + wt;
+      const uint32_t base = smem_u32(sW) + wt * 4;
+      // CTA `split` reduces rows m = split, split + S, ... in slice order
+      for (int m = split; m < p.M; m += p.splits) {
+        float acc = 0.0f;
+        for (int s = 0; s < p.splits; ++s)
+          acc = __fadd_rn(acc, ld_peer_f32(base + m * FBM * 4, static_cast<uint32_t>(s)));
+        if (n < p.N) store_out(p, m, n, __fmul_rn(alpha, acc));
+      }
+    }
+    // peers read this CTA's shared memory until here
+    cluster_sync_all();
   }
 
   tc_fence_before();
@@ -516,7 +573,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, F_TMEM_COLS);
+    tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
   }
 }
 
@@ -549,21 +606,28 @@ bool make_w_map(CUtensorMap* m, const uint8_t* base, int N, int K) {
 
 }  // namespace
 
+bool fused_supported(int M, int N, int K) {
+  if (M < 1 || M > 32 || N < 1 || K < 1) return false;
+  return make_plan(M, N, K).ok;
+}
+
 size_t fused_workspace_bytes(int M, int N, int K, int fmt) {
-  return make_plan(M, N, K, fmt).ws_bytes;
+  (void)M;
+  (void)N;
+  (void)K;
+  (void)fmt;
+  return align256(static_cast<size_t>(kMaxPrologueCtas) * sizeof(unsigned));
 }
 
 cudaError_t launch_gemm_fused(const FusedArgs& f, cudaStream_t s) {
-  const Plan pl = make_plan(f.M, f.N, f.K, f.fmt);
-  uint8_t* ws = static_cast<uint8_t*>(f.ws);
+  const Plan pl = make_plan(f.M, f.N, f.K);
+  if (!pl.ok) return cudaErrorInvalidValue;
   FParams p{};
   p.a = static_cast<const uint16_t*>(f.a);
   p.w_scales = f.w_scales;
   p.g_w = f.g_w;
   p.g_a = f.g_a;
-  p.amax_partial = reinterpret_cast<unsigned*>(ws + pl.ws_partial_off);
-  p.counters = reinterpret_cast<unsigned*>(ws + pl.ws_counter_off);
-  p.sums = reinterpret_cast<float*>(ws + pl.ws_sum_off);
+  p.amax_partial = static_cast<const unsigned*>(f.ws);
   p.C = f.C;
   p.ldc = f.ldc;
   p.M = f.M;
@@ -576,38 +640,63 @@ cudaError_t launch_gemm_fused(const FusedArgs& f, cudaStream_t s) {
   p.splits = pl.splits;
   p.steps_max = pl.steps_max;
   p.nmma_n = pl.nmma_n;
+  p.tmem_cols = pl.tmem_cols;
+  p.group = pl.group;
   p.ncb = ncb_of(nsf_of(f.K, f.fmt));
   p.watchdog = watchdog_ptr();
   if (!p.watchdog) return cudaErrorInvalidSymbol;
 
-  const long long n_vec = static_cast<long long>(f.M) * f.K / 8;
-  int pro_blocks = static_cast<int>(std::min<long long>(
-      kMaxPrologueCtas, std::max<long long>(1, (n_vec + kPrologueThreads * 4 - 1) /
-                                                   (kPrologueThreads * 4))));
-  pro_blocks = std::max(pro_blocks, (pl.n_tiles + kPrologueThreads - 1) / kPrologueThreads);
-  pro_blocks = std::min(pro_blocks, kMaxPrologueCtas);
-  p.n_partial = pro_blocks;
-  fused_prologue_kernel<<<pro_blocks, kPrologueThreads, 0, s>>>(
-      static_cast<const uint4*>(f.a), n_vec, f.dynamic, const_cast<unsigned*>(p.amax_partial),
-      p.counters, pl.n_tiles);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  if (f.dynamic) {
+    const long long n_vec = static_cast<long long>(f.M) * f.K / 8;
+    const int blocks = static_cast<int>(std::min<long long>(
+        kMaxPrologueCtas,
+        std::max<long long>(1, (n_vec + kPrologueThreads * 2 - 1) / (kPrologueThreads * 2))));
+    p.n_partial = blocks;
+    cudaLaunchConfig_t pc{};
+    pc.gridDim = dim3(static_cast<unsigned>(blocks));
+    pc.blockDim = dim3(kPrologueThreads);
+    pc.stream = s;
+    cudaLaunchAttribute pa[1];
+    pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pa[0].val.programmaticStreamSerializationAllowed = 1;
+    pc.attrs = pa;
+    pc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&pc, fused_amax_kernel, static_cast<const uint4*>(f.a), n_vec,
+                           static_cast<unsigned*>(f.ws));
+    if (e != cudaSuccess) return e;
+  }
 
   CUtensorMap mw;
   if (!make_w_map(&mw, f.w_codes, f.N, f.K)) return cudaErrorInvalidValue;
   auto kern = (f.fmt == 0) ? fused_kernel<0> : fused_kernel<1>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem_bytes);
   if (e != cudaSuccess) return e;
+  if (pl.splits > 1) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.n_tiles * pl.splits));
   cfg.blockDim = dim3(kFusedThreads);
   cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem_bytes);
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pl.splits > 1) {
+    // the S slices of a weight tile form one cluster and reduce through
+    // distributed shared memory
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(pl.splits);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  cfg.attrs = na ? attr : nullptr;
+  cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, kern, mw, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

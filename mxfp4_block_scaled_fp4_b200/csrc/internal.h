@@ -22,8 +22,11 @@ inline long long rows_pad128(long long rows) { return (rows + 127) / 128 * 128; 
 
 // amax over a bf16 tensor of n elements (n % 8 == 0): writes one partial
 // maximum (bf16 magnitude bits) per CTA into `partial`; *n_used = CTAs.
+// pdl: launch as a programmatic dependent of the previous kernel (the
+// kernels release their own dependents at once and wait for their
+// predecessor before reading their input).
 cudaError_t launch_amax(const void* x, long long n, unsigned* partial, int* n_used,
-                        cudaStream_t s);
+                        cudaStream_t s, bool pdl = false);
 
 struct QuantArgs {
   const void* x;        // bf16 [rows, K]
@@ -38,7 +41,7 @@ struct QuantArgs {
   uint8_t* codes;
   uint8_t* scales;
 };
-cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s);
+cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl = false);
 
 struct GemmArgs {
   const uint8_t* a_codes; const uint8_t* a_scales; const float* g_a;
@@ -57,6 +60,8 @@ struct FusedArgs {
   void* ws; size_t ws_bytes;
 };
 size_t fused_workspace_bytes(int M, int N, int K, int fmt);
+// Shapes the fused path takes: 1 <= M <= 32 and K up to 8 slices of 8192.
+bool fused_supported(int M, int N, int K);
 cudaError_t launch_gemm_fused(const FusedArgs& a, cudaStream_t s);
 
 }  // namespace fp4

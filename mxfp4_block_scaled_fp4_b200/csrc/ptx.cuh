@@ -164,6 +164,17 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 }
 constexpr uint32_t kLayoutSwizzle128B = 2;
 
+// Copy a 32-row x 16-byte block from shared memory into tensor memory at
+// columns [taddr, taddr + 4), replicated into all four 32-lane quarters.
+// It runs in the MMA pipe, ordered before the MMAs the same thread issues
+// after it (and, as measured on B200, stalling them): use it only where the
+// tensor pipe has slack.
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+               ::"r"(taddr), "l"(sdesc) : "memory");
+}
+constexpr uint32_t kLayoutNone = 0;
+
 // D (+)= A . B^T with per-16-element E4M3 scales (NVFP4 blocks).
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t sfa_tmem,
