@@ -247,6 +247,35 @@ def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak):
     return res
 
 
+def measure_decoder(torch, dev, batch_sizes=(1, 16, 256), reps=20):
+    """The synthetic 24-layer decoder (288 W4A4 GEMM calls per forward) and
+    the same forward in torch bf16, each captured once as a CUDA graph."""
+    from mxfp4_block_scaled_fp4_b200.decoder import SyntheticDecoder
+    dec = SyntheticDecoder(dev)
+    res = []
+    for M in batch_sizes:
+        x = torch.randn(M, 2880, generator=torch.Generator().manual_seed(M)).to(torch.bfloat16).to(dev)
+        row = {"M": M, "gemm_calls": 288}
+        for name, fn in (("fp4", dec.forward_fp4), ("bf16", dec.forward_bf16)):
+            g, _ = dec.capture(fn, x)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize(dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            row[f"us_per_forward_{name}"] = round(e0.elapsed_time(e1) * 1e3 / reps, 1)
+            del g
+        row["speedup_vs_bf16"] = round(row["us_per_forward_bf16"] / row["us_per_forward_fp4"], 3)
+        row["fp4_weight_bytes"] = dec.weight_bytes()
+        res.append(row)
+    return res
+
+
 def run_part(args, rank):
     """One supplementary measurement alone (profiling aid)."""
     import torch
@@ -261,6 +290,8 @@ def run_part(args, rank):
         if args.decode_shape:
             shapes = [tuple(int(v) for v in args.decode_shape.split(","))]
         line["decode"] = measure_decode(torch, ops, L, inputs, dev, peaks["hbm_gbs"], shapes)
+    elif args.only == "decoder":
+        line["decoder"] = measure_decoder(torch, dev)
     else:
         line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"])
     if rank == 0:
@@ -295,7 +326,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-suite", action="store_true",
                     help="skip the decode and quantize-sweep measurements")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quantize"],
+    ap.add_argument("--only", default="all",
+                    choices=["all", "prefill", "decode", "quantize", "decoder"],
                     help="run one part only (profiling); the JSON line then carries that part")
     ap.add_argument("--decode-shape", default=None, help="M,N,K: restrict the decode part")
     ap.add_argument("--shape", default=None,
@@ -312,7 +344,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank)
-    if args.only in ("decode", "quantize"):
+    if args.only in ("decode", "quantize", "decoder"):
         return run_part(args, rank)
     if args.warmup < 3:
         args.warmup = 3
@@ -460,6 +492,7 @@ def main():
     if not args.no_suite:
         line["decode"] = measure_decode(torch, ops, L, inputs, dev, peaks["hbm_gbs"])
         line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"])
+        line["decoder"] = measure_decoder(torch, dev)
         line["gpu_launches_note"] = ("gpu_launches counts the timed prefill steps only; the "
                                      "decode and sweep objects are timed separately")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
