@@ -444,6 +444,10 @@ cudaError_t launch_gemm_fused(const FusedArgs& f, cudaStream_t s) {
   q.g = f.g_a;
   q.codes = x_codes;
   q.scales = x_scales;
+  // scale columns past K of real rows are still zeroed (they meet zero codes,
+  // and 0 x NaN would not be 0); rows >= M only reach output columns that
+  // are never stored
+  q.zero_pad_rows = 0;
   cudaError_t e;
   if (f.dynamic) {
     int used = 0;

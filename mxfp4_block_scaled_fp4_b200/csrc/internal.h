@@ -40,6 +40,9 @@ struct QuantArgs {
   int n_partial;
   uint8_t* codes;
   uint8_t* scales;
+  // MMA layout: also zero the scales of rows [rows, rows rounded up to 128).
+  // The small-M GEMM never reads those rows' scales, so its chain skips it.
+  int zero_pad_rows = 1;
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl = false);
 

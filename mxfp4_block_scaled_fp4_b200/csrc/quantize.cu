@@ -238,7 +238,7 @@ cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl) {
   long long pad_a = 0, pad_b = 0;
   if (a.layout == 0) {
     pad_a = a.rows * (4 * ncb - nsf);
-    pad_b = (rows_pad128(a.rows) - a.rows) * 4 * ncb;
+    pad_b = a.zero_pad_rows ? (rows_pad128(a.rows) - a.rows) * 4 * ncb : 0;
   }
   const long long want = std::max((units + kThreads * 4 - 1) / (kThreads * 4),
                                   (pad_a + pad_b + kThreads - 1) / kThreads);
