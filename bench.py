@@ -38,6 +38,10 @@ WORKLOAD = "prefill W4A4 NVFP4 GEMM M=8192 N=28672 K=8192, bf16 out, activation 
 # amax pass reads 2 B; quantize pass reads 2 B, writes 0.5 B codes + 1/16 B scales
 QUANT_BYTES_PER_ELEM = 2.0 + 2.0 + 0.5 + 1.0 / 16.0
 FP4_OVER_BF16 = 4.0     # nominal dense FP4 / dense BF16 tensor throughput on B200 (9 / 2.25)
+# DRAM read + write bytes of one gemm_kernel launch on the bench shape, from a
+# one-pass ncu capture (profiles/gemm_kernel_8192x28672x8192_dram_traffic.md).
+# Set to None whenever gemm_kernel changes, until it is captured again.
+GEMM_TRAFFIC_BYTES = 566.8e6 + 430.5e6
 
 
 def load_peaks():
@@ -475,7 +479,9 @@ def main():
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (A 128 MiB, packed W 131 MiB, C 448 MiB)"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
-                     "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
+                     "traffic": GEMM_TRAFFIC_BYTES if (M, N, K) == (8192, 28672, 8192) else None,
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read + write)",
                      "kernel": "fp4 gemm_kernel (tcgen05 kind::mxf4nvf4)",
                      "peak_source": f"{src} bf16_tflops_sustained x {FP4_OVER_BF16:g} "
                                     "(nominal dense FP4/BF16 ratio)"},

@@ -183,6 +183,14 @@ fp4_status_t fp4_quantize_act_noalloc(const void* x, int rows, int K, fp4_format
  * raw word (0 = no timeout).  Returns FP4_ERR_DEVICE_TIMEOUT if it was set. */
 fp4_status_t fp4_device_status(unsigned* code, void* stream);
 
+/* Self-test of the failure detection (the pages have no counterpart): one
+ * kernel waits on a device barrier that nothing signals, with a bounded wait
+ * of limit_ns (0 < limit_ns <= 1 s), then sets the watchdog word and
+ * returns, as every kernel of this library does when one of its waits runs
+ * out.  A following fp4_device_status returns FP4_ERR_DEVICE_TIMEOUT and the
+ * CUDA context stays usable.  Nothing is faulted, trapped or hung. */
+fp4_status_t fp4_watchdog_selftest(unsigned long long limit_ns, void* stream);
+
 /* A static string naming the status (never NULL). */
 const char* fp4_status_string(fp4_status_t status);
 

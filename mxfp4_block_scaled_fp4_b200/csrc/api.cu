@@ -7,6 +7,7 @@
 
 #include "fp4.h"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace fp4 {
 
@@ -23,6 +24,20 @@ unsigned* watchdog_ptr() {
     cached[dev] = static_cast<unsigned*>(p);
   }
   return cached[dev];
+}
+
+// The watchdog self-test: one warp waits on an mbarrier that nothing
+// arrives on, with a bounded wait of limit_ns, and returns.
+__global__ void watchdog_selftest_kernel(unsigned* wd, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, wd, WD_SELFTEST, limit_ns);
 }
 
 }  // namespace fp4
@@ -211,6 +226,16 @@ fp4_status_t fp4_gemm_fused(const void* x, const uint8_t* w_codes, const uint8_t
   a.ws = ws;
   a.ws_bytes = ws_bytes;
   return from_cuda(fp4::launch_gemm_fused(a, static_cast<cudaStream_t>(stream)));
+}
+
+fp4_status_t fp4_watchdog_selftest(unsigned long long limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return FP4_ERR_INVALID_ARG;
+  fp4_status_t st;
+  if ((st = device_ok()) != FP4_OK) return st;
+  unsigned* wd = fp4::watchdog_ptr();
+  if (!wd) return FP4_ERR_CUDA;
+  fp4::watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(wd, limit_ns);
+  return from_cuda(cudaGetLastError());
 }
 
 fp4_status_t fp4_device_status(unsigned* code, void* stream) {

@@ -16,6 +16,7 @@ enum : unsigned {
   WD_EPILOGUE = 1u << 3,   // epilogue waited too long for the accumulator
   WD_DRAIN    = 1u << 4,   // in-flight copies did not land during unwinding
   WD_STAGING  = 1u << 5,   // scale-staging warps waited too long for a loaded stage
+  WD_SELFTEST = 1u << 6,   // the watchdog self-test's wait ran out (expected)
 };
 
 // Time budget of one wait (ns).  Legitimate waits here are microseconds.
@@ -61,10 +62,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for phase `parity` of `bar` to complete.  Gives up (returns false)
-// when *abort is raised by another role or after kWaitLimitNs, in which
-// case it records `code` in the watchdog word and raises *abort.
+// when *abort is raised by another role or after limit_ns, in which case it
+// records `code` in the watchdog word and raises *abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort, unsigned* wd, unsigned code) {
+                                          volatile int* abort, unsigned* wd, unsigned code,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
@@ -72,7 +74,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 15u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         atomicOr(wd, code);
         *abort = 1;
         return false;

@@ -62,6 +62,7 @@ SIGNATURES = {
     "fp4_gemm_fused": (I, [P, U8P, U8P, FP, I, I, I, I, I, FP, P, I, I, P, SZ, P]),
     "fp4_quantize_act_noalloc": (I, [P, I, I, I, I, I, FP, U8P, U8P, P]),
     "fp4_device_status": (I, [ctypes.POINTER(ctypes.c_uint), P]),
+    "fp4_watchdog_selftest": (I, [ctypes.c_ulonglong, P]),
     "fp4_status_string": (ctypes.c_char_p, [I]),
 }
 
@@ -137,6 +138,10 @@ def fp4_device_status(stream=None):
     code = ctypes.c_uint(0)
     st = _call("fp4_device_status", ctypes.byref(code), stream)
     return st, code.value
+
+
+def fp4_watchdog_selftest(limit_ns, stream=None):
+    return _call("fp4_watchdog_selftest", limit_ns, stream)
 
 
 def fp4_status_string(status):
