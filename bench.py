@@ -38,9 +38,9 @@ WORKLOAD = "prefill W4A4 NVFP4 GEMM M=8192 N=28672 K=8192, bf16 out, activation 
 # amax pass reads 2 B; quantize pass reads 2 B, writes 0.5 B codes + 1/16 B scales
 QUANT_BYTES_PER_ELEM = 2.0 + 2.0 + 0.5 + 1.0 / 16.0
 FP4_OVER_BF16 = 4.0     # nominal dense FP4 / dense BF16 tensor throughput on B200 (9 / 2.25)
-# DRAM read + write bytes of one gemm_kernel launch on the bench shape, from a
-# one-pass ncu capture (profiles/gemm_kernel_8192x28672x8192_dram_traffic.md).
-# Set to None whenever gemm_kernel changes, until it is captured again.
+# DRAM read + write bytes of one gemm_kernel launch on the bench shape,
+# measured with ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass).
+# Set to None whenever gemm_kernel changes, until it is measured again.
 GEMM_TRAFFIC_BYTES = 566.8e6 + 430.5e6
 
 
