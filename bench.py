@@ -38,10 +38,11 @@ WORKLOAD = "prefill W4A4 NVFP4 GEMM M=8192 N=28672 K=8192, bf16 out, activation 
 # amax pass reads 2 B; quantize pass reads 2 B, writes 0.5 B codes + 1/16 B scales
 QUANT_BYTES_PER_ELEM = 2.0 + 2.0 + 0.5 + 1.0 / 16.0
 FP4_OVER_BF16 = 4.0     # nominal dense FP4 / dense BF16 tensor throughput on B200 (9 / 2.25)
-# DRAM read + write bytes of one gemm_kernel launch on the bench shape,
-# measured with ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass).
-# Set to None whenever gemm_kernel changes, until it is measured again.
-GEMM_TRAFFIC_BYTES = 566.8e6 + 430.5e6
+# DRAM read + write bytes of one launch of the GEMM kernel the bench shape
+# takes (gemm_pair_kernel), measured with ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum, one pass).  None whenever that kernel has changed
+# since it was last measured.
+GEMM_TRAFFIC_BYTES = None
 
 
 def load_peaks():
@@ -482,7 +483,7 @@ def main():
                      "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
                      "traffic": GEMM_TRAFFIC_BYTES if (M, N, K) == (8192, 28672, 8192) else None,
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read + write)",
-                     "kernel": "fp4 gemm_kernel (tcgen05 kind::mxf4nvf4)",
+                     "kernel": "fp4 gemm_pair_kernel (tcgen05 cta_group::2 kind::mxf4nvf4)",
                      "peak_source": f"{src} bf16_tflops_sustained x {FP4_OVER_BF16:g} "
                                     "(nominal dense FP4/BF16 ratio)"},
         "quantize": {"achieved_gbs": q_gbs, "peak_gbs": peaks["hbm_gbs"],

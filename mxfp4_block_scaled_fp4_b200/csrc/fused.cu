@@ -114,10 +114,6 @@ __device__ __forceinline__ void grid_dep_launch() {
 __device__ __forceinline__ void workers_sync() {   // named barrier of the 4 worker warps
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
 __device__ __forceinline__ float ld_peer_f32(uint32_t local_saddr, uint32_t rank) {
   uint32_t remote;
   float v;

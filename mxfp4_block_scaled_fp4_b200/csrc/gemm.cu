@@ -384,9 +384,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Packed FP4 codes [rows, K/2] bytes viewed as a 2-D uint8 tensor; the box
-// is 128 bytes of K by box_rows rows with 128-byte swizzle.  Out-of-range
-// rows and columns read as zero codes.
+}  // namespace
+
 bool make_code_map(CUtensorMap* m, const uint8_t* base, long long rows, int K, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -399,6 +398,8 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, long long rows, int K, i
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int FMT, int OUT_F32>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const Params& p, int grid,
@@ -413,6 +414,7 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const Par
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  if (a.M > BM) return launch_gemm_pair(a, s);
   CUtensorMap ma, mw;
   if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, a.w_codes, a.N, a.K, BN)) return cudaErrorInvalidValue;

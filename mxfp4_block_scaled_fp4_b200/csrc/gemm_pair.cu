@@ -1,0 +1,497 @@
+// gemm_pair.cu -- the block-scaled FP4 GEMM of gemm.cu on CTA pairs
+// (tcgen05 cta_group::2), used when M > 128.
+//
+//   C[M, N] = alpha * sum_k s_a[m, k/B] q_a[m, k] * s_w[n, k/B] q_w[n, k]
+//
+// (the W4A4 GEMM of the "fp4-cuda-kernel" forum post; NVFP4 / MXFP4 block
+// formats as in gemm.cu.)
+//
+// The output is cut into 256 x 256 tiles, each computed by a cluster of two
+// CTAs on the two SMs of a TPC.  CTA r of the pair holds rows r*128 .. +127
+// of the tile's A slice and of its W slice in its own shared memory; one
+// tcgen05.mma (M = 256, N = 256, K = 64) issued by the even CTA (the leader)
+// reads A from each CTA's own half and W from both halves, and leaves
+// accumulator rows r*128 .. +127 (all 256 columns) in CTA r's tensor memory,
+// next to CTA r's own copy of the scales.  Per SM and per MMA that halves the
+// W bytes loaded into and read out of shared memory compared with the
+// one-CTA 128 x 256 tile (12 KiB -> 8 KiB of operand traffic per 128 x 256 x
+// 64 step); measured on B200 it is 8-13% faster than the one-CTA kernel on
+// large prefill shapes and bit-identical to it.
+//
+// Roles (10 warps in each CTA of the pair):
+//   warp 0      TMA for this CTA: its A and W halves (plain, non-multicast
+//               tiled loads onto its own `full` barrier) and its scale atoms
+//               (the A row block of its half; both W row blocks of the tile,
+//               which every SM's MMA reads from its own tensor memory);
+//   warp 1      both CTAs: tensor-memory allocation for the pair; leader,
+//               one thread: issues the pair MMAs, commits to both CTAs'
+//               `empty` / `acc_full` barriers (multicast commit);
+//   warps 2-5   epilogue of this CTA's 128 accumulator rows, then release
+//               the accumulator on the leader's `acc_empty` (count 8);
+//   warps 6-9   scale staging into this CTA's tensor memory with tcgen05.st;
+//               once the stage's code tiles have landed as well, each warp
+//               arrives on the leader's `ready` barrier (count 8), so the MMA
+//               thread waits on one barrier for both CTAs' data.
+// The hand-offs between the CTAs are plain remote mbarrier arrivals: what
+// they publish is ordered by tcgen05.wait::st / tcgen05.ld waits and the
+// tcgen05 thread-sync fences (tensor memory) or by an mbarrier the arriving
+// warp has itself observed complete (shared memory written by TMA).  A
+// release at cluster scope on the per-stage arrival was measured to cost
+// ~1000 cycles per K step and to halve the kernel's speed.
+// Every copy is issued and awaited by the CTA whose shared memory it fills,
+// so on an abort each CTA drains its own copies.  Every wait is bounded; a
+// wait that runs out sets the watchdog word and raises the abort flag of
+// both CTAs, the leader waits for its MMAs in flight, and both CTAs meet at
+// a final cluster barrier before the pair's tensor memory is freed.
+#include <algorithm>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fp4 {
+
+namespace {
+
+constexpr int BM = 256;                 // tile rows (128 per CTA)
+constexpr int BN = 256;                 // tile columns (128 W rows per CTA)
+constexpr int HALF = 128;
+constexpr int BK = 256;
+constexpr int BK_BYTES = BK / 2;
+constexpr int MMA_K = 64;
+constexpr int STAGES = 5;
+constexpr int A_STAGE = HALF * BK_BYTES;   // 16 KiB
+constexpr int B_STAGE = HALF * BK_BYTES;   // 16 KiB
+constexpr int SFA_STAGE = 4 * 512;
+constexpr int SFB_STAGE = 2 * 4 * 512;
+constexpr int RING_BYTES = STAGES * (A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE);
+constexpr int SMEM_BYTES = RING_BYTES + 1024 + 256;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;
+constexpr uint32_t SF_COL = 256;
+constexpr uint32_t SF_STAGE_COLS = 48;
+constexpr int kThreads = 320;
+constexpr int GROUP_M = 16;             // raster: 16 tile rows (4096 rows of A) share W in L2
+
+static_assert(SF_COL + STAGES * SF_STAGE_COLS <= TMEM_COLS, "scale stages exceed tensor memory");
+static_assert(SMEM_BYTES <= 227 * 1024, "ring exceeds shared memory");
+
+struct Params {
+  const uint8_t* a_scales;
+  const uint8_t* w_scales;
+  const float* g_a;
+  const float* g_w;
+  void* C;
+  long long ldc;
+  int M, N, K;
+  int m_tiles, n_tiles, k_steps;
+  int ncb;
+  int a_rowblocks;        // ceil(M / 128)
+  int w_rowblocks;        // ceil(N / 128)
+  unsigned* watchdog;
+};
+
+__device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int& nt) {
+  const int per_group = GROUP_M * p.n_tiles;
+  const int group = t / per_group;
+  const int first_m = group * GROUP_M;
+  const int gsize = min(GROUP_M, p.m_tiles - first_m);
+  const int within = t - group * per_group;
+  mt = first_m + within % gsize;
+  nt = within / gsize;
+}
+
+template <int FMT, int OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
+                     const __grid_constant__ CUtensorMap tm_w, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  // the same 1024-aligned offset in both CTAs: the pair MMA addresses the
+  // peer's operands with this CTA's descriptors
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_STAGE;
+  uint8_t* sSFA = sB + STAGES * B_STAGE;
+  uint8_t* sSFB = sSFA + STAGES * SFA_STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_STAGE);
+  uint64_t* sf_loaded = full + STAGES;
+  uint64_t* empty = sf_loaded + STAGES;
+  uint64_t* ready = empty + STAGES;
+  uint64_t* acc_full = ready + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&sf_loaded[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&ready[s], 8);     // 4 staging warps in each CTA of the pair
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);       // 4 epilogue warps in each CTA of the pair
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tm_a);
+    prefetch_tensormap(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  // barriers initialised and tensor memory allocated in both CTAs before any
+  // remote arrival
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t peer_abort = map_to_rank(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
+
+  const int n_tiles_total = p.m_tiles * p.n_tiles;
+  const int first = static_cast<int>(cluster_id_x());
+  const int stride = static_cast<int>(nclusters_x());
+  constexpr int kAtomsPerStage = (FMT == 0) ? 4 : 2;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0, armed_parity = 0;
+    for (int t = first; t < n_tiles_total; t += stride) {
+      int mt, nt;
+      tile_coords(t, p, mt, nt);
+      const int rba = mt * 2 + static_cast<int>(rank);   // A row block of this CTA's half
+      const bool a_rows = rba < p.a_rowblocks;
+      const int rb0 = nt * 2;
+      const int wblocks = min(2, p.w_rowblocks - rb0);
+      for (int kb = 0; kb < p.k_steps; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.watchdog, WD_PRODUCER)) {
+          st_cluster_u32(peer_abort, 1u);
+          goto producer_drain;
+        }
+        {
+          const int cb0 = kb * kAtomsPerStage;
+          const int atoms = min(kAtomsPerStage, p.ncb - cb0);
+          const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
+          // a half made only of rows past M has no scale atoms; its
+          // accumulator rows are never stored
+          mbar_expect_tx(&sf_loaded[stage], sf_bytes * ((a_rows ? 1 : 0) + wblocks));
+          if (a_rows)
+            bulk_load(sSFA + stage * SFA_STAGE,
+                      p.a_scales + (static_cast<long long>(rba) * p.ncb + cb0) * 512, sf_bytes,
+                      &sf_loaded[stage]);
+          for (int i = 0; i < wblocks; ++i)
+            bulk_load(sSFB + stage * SFB_STAGE + i * 2048,
+                      p.w_scales + (static_cast<long long>(rb0 + i) * p.ncb + cb0) * 512, sf_bytes,
+                      &sf_loaded[stage]);
+          mbar_expect_tx(&full[stage], A_STAGE + B_STAGE);
+          tma_load_2d(sA + stage * A_STAGE, &tm_a, kb * BK_BYTES, mt * BM + rank * HALF,
+                      &full[stage]);
+          tma_load_2d(sB + stage * B_STAGE, &tm_w, kb * BK_BYTES, nt * BN + rank * HALF,
+                      &full[stage]);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    goto producer_done;
+  producer_drain:
+    for (int s = 0; s < STAGES; ++s)
+      if (armed & (1u << s)) {
+        mbar_wait_drain(&sf_loaded[s], (armed_parity >> s) & 1u, p.watchdog);
+        mbar_wait_drain(&full[s], (armed_parity >> s) & 1u, p.watchdog);
+      }
+  producer_done:;
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------------------------------------------- pair MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    for (int t = first; t < n_tiles_total; t += stride, ++it) {
+      if (it > 0 && !mbar_wait(acc_empty, static_cast<uint32_t>(it - 1) & 1u, abort_flag,
+                                     p.watchdog, WD_MMA_ACC)) {
+        st_cluster_u32(peer_abort, 1u);
+        goto mma_drain;
+      }
+      tc_fence_after();
+      for (int kb = 0; kb < p.k_steps; ++kb) {
+        if (!mbar_wait(&ready[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) {
+          st_cluster_u32(peer_abort, 1u);
+          goto mma_drain;
+        }
+        tc_fence_after();
+        {
+          const int n_mma = min(BK / MMA_K, (p.K - kb * BK + MMA_K - 1) / MMA_K);
+          const uint32_t sfa_t = tmem + SF_COL + stage * SF_STAGE_COLS;
+          const uint32_t sfb_t = sfa_t + 16;
+          const uint32_t a_s = smem_u32(sA + stage * A_STAGE);
+          const uint32_t b_s = smem_u32(sB + stage * B_STAGE);
+          for (int k = 0; k < n_mma; ++k) {
+            const uint64_t ad = smem_desc(a_s + k * (MMA_K / 2), 16, 1024, kLayoutSwizzle128B);
+            const uint64_t bd = smem_desc(b_s + k * (MMA_K / 2), 16, 1024, kLayoutSwizzle128B);
+            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+            if (FMT == 0) {
+              tc_mma_pair_nvf4(tmem + ACC_COL, ad, bd, idesc_fp4(BM, BN, false, 0, 0),
+                               sfa_t + 4 * k, sfb_t + 8 * k, acc);
+            } else {
+              const uint32_t id = 2u * (k & 1);
+              tc_mma_pair_mxf4(tmem + ACC_COL, ad, bd, idesc_fp4(BM, BN, true, id, id),
+                               sfa_t + 4 * (k >> 1), sfb_t + 8 * (k >> 1), acc);
+            }
+          }
+        }
+        tc_commit_pair(&empty[stage], 0x3);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      tc_commit_pair(acc_full, 0x3);
+    }
+    goto mma_done;
+  mma_drain:
+    tc_commit_pair(drain, 0x1);
+    mbar_wait_drain(drain, 0, p.watchdog);
+  mma_done:;
+  } else if (warp >= 6) {
+    // ----------------------------------------------------- scale staging
+    const int quarter = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = first; t < n_tiles_total; t += stride) {
+      for (int kb = 0; kb < p.k_steps; ++kb) {
+        if (!__all_sync(0xFFFFFFFFu,
+                        mbar_wait(&sf_loaded[stage], phase, abort_flag, p.watchdog, WD_STAGING))) {
+          if (lane == 0) st_cluster_u32(peer_abort, 1u);
+          goto staging_done;
+        }
+        {
+          const uint32_t sfa_s = smem_u32(sSFA + stage * SFA_STAGE) + lane * 16;
+          const uint32_t sfb_s = smem_u32(sSFB + stage * SFB_STAGE) + lane * 16;
+          const uint32_t sfa_t = tmem + lane_off + SF_COL + stage * SF_STAGE_COLS;
+          const uint32_t sfb_t = sfa_t + 16;
+          uint32_t va[4 * kAtomsPerStage], vb[8 * kAtomsPerStage];
+#pragma unroll
+          for (int a = 0; a < kAtomsPerStage; ++a) {
+            const uint4 x = lds128(sfa_s + a * 512);
+            va[4 * a + 0] = x.x; va[4 * a + 1] = x.y; va[4 * a + 2] = x.z; va[4 * a + 3] = x.w;
+#pragma unroll
+            for (int rb = 0; rb < 2; ++rb) {
+              const uint4 y = lds128(sfb_s + rb * 2048 + a * 512);
+              vb[8 * a + 4 * rb + 0] = y.x; vb[8 * a + 4 * rb + 1] = y.y;
+              vb[8 * a + 4 * rb + 2] = y.z; vb[8 * a + 4 * rb + 3] = y.w;
+            }
+          }
+          if (kAtomsPerStage == 4) {
+            tmem_st_x16(sfa_t, va);
+            tmem_st_x32(sfb_t, vb);
+          } else {
+            tmem_st_x8(sfa_t, va);
+            tmem_st_x16(sfb_t, vb);
+          }
+          tmem_st_wait();
+        }
+        // the stage's code tiles must have landed in this CTA as well before
+        // the leader may issue the MMAs that read them
+        if (!__all_sync(0xFFFFFFFFu,
+                        mbar_wait(&full[stage], phase, abort_flag, p.watchdog, WD_STAGING))) {
+          if (lane == 0) st_cluster_u32(peer_abort, 1u);
+          goto staging_done;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(&ready[stage]);
+          else
+            mbar_arrive_remote(map_to_rank(smem_u32(&ready[stage]), 0));
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  staging_done:;
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    float alpha = 1.0f;
+    if (FMT == 0) alpha = __fmul_rn(*p.g_a, *p.g_w);
+    const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
+    int it = 0;
+    for (int t = first; t < n_tiles_total; t += stride, ++it) {
+      int mt, nt;
+      tile_coords(t, p, mt, nt);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag,
+                                             p.watchdog, WD_EPILOGUE))) {
+        if (lane == 0) st_cluster_u32(peer_abort, 1u);
+        break;
+      }
+      tc_fence_after();
+      const int row = mt * BM + static_cast<int>(rank) * HALF + quarter * 32 + lane;
+      const bool row_ok = row < p.M;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL;
+      if (!OUT_F32) {
+        uint32_t packed[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float lo = __fmul_rn(alpha, __uint_as_float(r[2 * j]));
+            const float hi = __fmul_rn(alpha, __uint_as_float(r[2 * j + 1]));
+            __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+            packed[16 * c + j] = *reinterpret_cast<uint32_t*>(&h);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(acc_empty);
+          else
+            mbar_arrive_remote(acc_empty_leader);
+        }
+        if (row_ok) {
+          uint16_t* out = static_cast<uint16_t*>(p.C) + static_cast<long long>(row) * p.ldc;
+#pragma unroll
+          for (int v = 0; v < BN / 8; ++v) {
+            const int n = nt * BN + 8 * v;
+            if (n < p.N)
+              *reinterpret_cast<uint4*>(out + n) = make_uint4(packed[4 * v], packed[4 * v + 1],
+                                                              packed[4 * v + 2], packed[4 * v + 3]);
+          }
+        }
+      } else {
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
+          tmem_ld_wait();
+          if (c == BN / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+          if (leader)
+            mbar_arrive(acc_empty);
+          else
+            mbar_arrive_remote(acc_empty_leader);
+        }
+          }
+          const int n0 = nt * BN + c * 32;
+          if (!row_ok || n0 >= p.N) continue;
+          float* out = static_cast<float*>(p.C) + static_cast<long long>(row) * p.ldc + n0;
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            if (n0 + 4 * v < p.N) {
+              float4 o;
+              o.x = __fmul_rn(alpha, __uint_as_float(r[4 * v + 0]));
+              o.y = __fmul_rn(alpha, __uint_as_float(r[4 * v + 1]));
+              o.z = __fmul_rn(alpha, __uint_as_float(r[4 * v + 2]));
+              o.w = __fmul_rn(alpha, __uint_as_float(r[4 * v + 3]));
+              *reinterpret_cast<float4*>(out + 4 * v) = o;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // neither CTA leaves (or frees tensor memory) while the other may still
+  // arrive on its barriers or the leader's MMAs may still touch its memory
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------ host side
+
+template <int FMT, int OUT_F32>
+cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const Params& p, int tiles,
+                         cudaStream_t s) {
+  auto kern = gemm_pair_kernel<FMT, OUT_F32>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // pairs that fit on the device at once (cached per device)
+  static int max_pairs[64] = {0};
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (max_pairs[dev] <= 0) {
+    cfg.gridDim = dim3(2);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n <= 0) return cudaErrorInvalidConfiguration;
+    max_pairs[dev] = n;
+  }
+  const int pairs = std::max(1, std::min(tiles, max_pairs[dev]));
+  cfg.gridDim = dim3(2 * pairs);
+  e = cudaLaunchKernelEx(&cfg, kern, ma, mw, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
+  CUtensorMap ma, mw;
+  if (!make_code_map(&ma, a.a_codes, a.M, a.K, HALF)) return cudaErrorInvalidValue;
+  if (!make_code_map(&mw, a.w_codes, a.N, a.K, HALF)) return cudaErrorInvalidValue;
+  Params p;
+  p.a_scales = a.a_scales;
+  p.w_scales = a.w_scales;
+  p.g_a = a.g_a;
+  p.g_w = a.g_w;
+  p.C = a.C;
+  p.ldc = a.ldc;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.m_tiles = (a.M + BM - 1) / BM;
+  p.n_tiles = (a.N + BN - 1) / BN;
+  p.k_steps = (a.K + BK - 1) / BK;
+  p.ncb = ncb_of(nsf_of(a.K, a.fmt));
+  p.a_rowblocks = (a.M + HALF - 1) / HALF;
+  p.w_rowblocks = (a.N + HALF - 1) / HALF;
+  p.watchdog = watchdog_ptr();
+  if (!p.watchdog) return cudaErrorInvalidSymbol;
+  const int tiles = p.m_tiles * p.n_tiles;
+  if (a.fmt == 0)
+    return a.out_f32 ? launch_typed<0, 1>(ma, mw, p, tiles, s) : launch_typed<0, 0>(ma, mw, p, tiles, s);
+  return a.out_f32 ? launch_typed<1, 1>(ma, mw, p, tiles, s) : launch_typed<1, 0>(ma, mw, p, tiles, s);
+}
+
+}  // namespace fp4

@@ -1,5 +1,6 @@
 // internal.h -- launchers shared between the C-ABI layer and the kernels.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -53,6 +54,13 @@ struct GemmArgs {
   void* C; int ldc; int out_f32;
 };
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s);
+// The CTA-pair kernel (256-row tiles); launch_gemm takes it for M > 128.
+cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s);
+
+// Tensor map of packed FP4 codes [rows, K/2] bytes as a 2-D uint8 tensor:
+// box of 128 bytes of K by box_rows rows, 128-byte swizzle, out-of-range
+// rows and columns read as zero codes.
+bool make_code_map(CUtensorMap* m, const uint8_t* base, long long rows, int K, int box_rows);
 
 struct FusedArgs {
   const void* a;        // bf16 [M, K]

@@ -52,7 +52,7 @@ def test_pr1_tiny_outliers(ops, orc, fmt, dt, fused):
 
 
 RAGGED = [(1, 8, 32), (16, 256, 64), (130, 264, 2880), (300, 520, 1056), (257, 512, 4096),
-          (128, 256, 256), (129, 136, 96)]
+          (128, 256, 256), (129, 136, 96), (2304, 2312, 320)]
 
 
 @pytest.mark.parametrize("M,N,K", RAGGED)
