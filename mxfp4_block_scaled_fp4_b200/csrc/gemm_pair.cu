@@ -65,7 +65,11 @@ constexpr int B_STAGE = HALF * BK_BYTES;   // 16 KiB
 constexpr int SFA_STAGE = 4 * 512;
 constexpr int SFB_STAGE = 2 * 4 * 512;
 constexpr int RING_BYTES = STAGES * (A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE);
-constexpr int SMEM_BYTES = RING_BYTES + 1024 + 256;
+// bf16 epilogue staging: per epilogue warp two 32-row x 64-column buffers
+// (4 KiB each, 128-byte swizzle) that TMA stores drain to C
+constexpr int OUT_BUF = 32 * 128;
+constexpr int OUT_BYTES = 4 * 2 * OUT_BUF;
+constexpr int SMEM_BYTES = RING_BYTES + OUT_BYTES + 1024 + 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = 256;
@@ -75,6 +79,7 @@ constexpr int GROUP_M = 16;             // raster: 16 tile rows (4096 rows of A)
 
 static_assert(SF_COL + STAGES * SF_STAGE_COLS <= TMEM_COLS, "scale stages exceed tensor memory");
 static_assert(SMEM_BYTES <= 227 * 1024, "ring exceeds shared memory");
+static_assert(RING_BYTES % 1024 == 0, "epilogue buffers must stay 1024-byte aligned");
 
 struct Params {
   const uint8_t* a_scales;
@@ -104,7 +109,8 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int
 template <int FMT, int OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
-                     const __grid_constant__ CUtensorMap tm_w, const Params p) {
+                     const __grid_constant__ CUtensorMap tm_w,
+                     const __grid_constant__ CUtensorMap tm_c, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   // the same 1024-aligned offset in both CTAs: the pair MMA addresses the
   // peer's operands with this CTA's descriptors
@@ -114,7 +120,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sB = sA + STAGES * A_STAGE;
   uint8_t* sSFA = sB + STAGES * B_STAGE;
   uint8_t* sSFB = sSFA + STAGES * SFA_STAGE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_STAGE);
+  uint8_t* sOut = sSFB + STAGES * SFB_STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_BYTES);
   uint64_t* sf_loaded = full + STAGES;
   uint64_t* empty = sf_loaded + STAGES;
   uint64_t* ready = empty + STAGES;
@@ -143,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_w);
+    if (!OUT_F32) prefetch_tensormap(&tm_c);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -217,47 +225,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   producer_done:;
   } else if (warp == 1 && lane == 0 && leader) {
     // ---------------------------------------------------- pair MMA issuer
+    // Lean loop: the pipe runs one 256 x 256 x 64 MMA per 128 cycles and an
+    // issue costs this thread ~75, so everything else it does between two
+    // K steps must fit in ~200 cycles or the pipe idles (measured on B200).
+    // Descriptors advance by adding to their address field; the next
+    // stage's `ready` is polled while this stage's MMAs are queued.
+    const uint64_t a_desc0 = smem_desc(smem_u32(sA), 16, 1024, kLayoutSwizzle128B);
+    const uint64_t b_desc0 = smem_desc(smem_u32(sB), 16, 1024, kLayoutSwizzle128B);
+    const uint32_t ready0 = smem_u32(ready);
+    const uint32_t sf0 = tmem + SF_COL;
+    constexpr uint32_t kIdesc0 = idesc_fp4(BM, BN, FMT == 1, 0, 0);
+    constexpr uint32_t kIdesc2 = idesc_fp4(BM, BN, FMT == 1, 2, 2);
+    // MMAs in the last K step (K may end inside it)
+    const int last_mmas = (p.K - (p.k_steps - 1) * BK + MMA_K - 1) / MMA_K;
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
+    bool next_ready = false;
     for (int t = first; t < n_tiles_total; t += stride, ++it) {
       if (it > 0 && !mbar_wait(acc_empty, static_cast<uint32_t>(it - 1) & 1u, abort_flag,
-                                     p.watchdog, WD_MMA_ACC)) {
+                               p.watchdog, WD_MMA_ACC)) {
         st_cluster_u32(peer_abort, 1u);
         goto mma_drain;
       }
       tc_fence_after();
       for (int kb = 0; kb < p.k_steps; ++kb) {
-        if (!mbar_wait(&ready[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) {
+        if (!next_ready && !mbar_try_wait(ready0 + stage * 8, phase) &&
+            !mbar_wait(&ready[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) {
           st_cluster_u32(peer_abort, 1u);
           goto mma_drain;
         }
         tc_fence_after();
+        int nstage = stage + 1;
+        uint32_t nphase = phase;
+        if (nstage == STAGES) {
+          nstage = 0;
+          nphase ^= 1u;
+        }
+        const bool has_next = kb + 1 < p.k_steps;
+        next_ready = false;
         {
-          const int n_mma = min(BK / MMA_K, (p.K - kb * BK + MMA_K - 1) / MMA_K);
-          const uint32_t sfa_t = tmem + SF_COL + stage * SF_STAGE_COLS;
+          const int n_mma = has_next ? BK / MMA_K : last_mmas;
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>(stage * (A_STAGE >> 4));
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>(stage * (B_STAGE >> 4));
+          const uint32_t sfa_t = sf0 + stage * SF_STAGE_COLS;
           const uint32_t sfb_t = sfa_t + 16;
-          const uint32_t a_s = smem_u32(sA + stage * A_STAGE);
-          const uint32_t b_s = smem_u32(sB + stage * B_STAGE);
-          for (int k = 0; k < n_mma; ++k) {
-            const uint64_t ad = smem_desc(a_s + k * (MMA_K / 2), 16, 1024, kLayoutSwizzle128B);
-            const uint64_t bd = smem_desc(b_s + k * (MMA_K / 2), 16, 1024, kLayoutSwizzle128B);
-            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-            if (FMT == 0) {
-              tc_mma_pair_nvf4(tmem + ACC_COL, ad, bd, idesc_fp4(BM, BN, false, 0, 0),
-                               sfa_t + 4 * k, sfb_t + 8 * k, acc);
-            } else {
-              const uint32_t id = 2u * (k & 1);
-              tc_mma_pair_mxf4(tmem + ACC_COL, ad, bd, idesc_fp4(BM, BN, true, id, id),
-                               sfa_t + 4 * (k >> 1), sfb_t + 8 * (k >> 1), acc);
+#pragma unroll
+          for (int k = 0; k < BK / MMA_K; ++k) {
+            if (k < n_mma) {
+              // 32 bytes of K per MMA = 2 units of the descriptor's address field
+              const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+              if (FMT == 0)
+                tc_mma_pair_nvf4(tmem + ACC_COL, ad + 2 * k, bd + 2 * k, kIdesc0, sfa_t + 4 * k,
+                                 sfb_t + 8 * k, acc);
+              else
+                tc_mma_pair_mxf4(tmem + ACC_COL, ad + 2 * k, bd + 2 * k,
+                                 (k & 1) ? kIdesc2 : kIdesc0, sfa_t + 4 * (k >> 1),
+                                 sfb_t + 8 * (k >> 1), acc);
             }
+            if (k == 1 && has_next) next_ready = mbar_try_wait(ready0 + nstage * 8, nphase);
           }
         }
         tc_commit_pair(&empty[stage], 0x3);
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        stage = nstage;
+        phase = nphase;
       }
       tc_commit_pair(acc_full, 0x3);
     }
@@ -333,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float alpha = 1.0f;
     if (FMT == 0) alpha = __fmul_rn(*p.g_a, *p.g_w);
     const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
+    uint8_t* sOutW = sOut + (warp - 2) * 2 * OUT_BUF;
     int it = 0;
     for (int t = first; t < n_tiles_total; t += stride, ++it) {
       int mt, nt;
@@ -369,14 +401,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             mbar_arrive_remote(acc_empty_leader);
         }
-        if (row_ok) {
-          uint16_t* out = static_cast<uint16_t*>(p.C) + static_cast<long long>(row) * p.ldc;
+        // C rows row0 .. row0+31 leave through this warp's two swizzled
+        // buffers and 64-column TMA stores (rows past M and columns past N
+        // are clipped by the store)
+        const int row0 = mt * BM + static_cast<int>(rank) * HALF + quarter * 32;
+        if (row0 < p.M) {
 #pragma unroll
-          for (int v = 0; v < BN / 8; ++v) {
-            const int n = nt * BN + 8 * v;
-            if (n < p.N)
-              *reinterpret_cast<uint4*>(out + n) = make_uint4(packed[4 * v], packed[4 * v + 1],
-                                                              packed[4 * v + 2], packed[4 * v + 3]);
+          for (int c = 0; c < BN / 64; ++c) {
+            const int n0 = nt * BN + 64 * c;
+            if (n0 < p.N) {
+              uint8_t* buf = sOutW + (c & 1) * OUT_BUF;
+              // the buffer's previous store must have finished reading it
+              if (lane == 0) bulk_wait_read_1();
+              __syncwarp();
+              const uint32_t rowaddr = smem_u32(buf) + lane * 128;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                sts128(rowaddr + ((j ^ (lane & 7)) << 4), packed[32 * c + 4 * j],
+                       packed[32 * c + 4 * j + 1], packed[32 * c + 4 * j + 2],
+                       packed[32 * c + 4 * j + 3]);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tm_c, buf, n0, row0);
+                bulk_commit();
+              }
+            }
           }
         }
       } else {
@@ -388,11 +438,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-          if (leader)
-            mbar_arrive(acc_empty);
-          else
-            mbar_arrive_remote(acc_empty_leader);
-        }
+              if (leader)
+                mbar_arrive(acc_empty);
+              else
+                mbar_arrive_remote(acc_empty_leader);
+            }
           }
           const int n0 = nt * BN + c * 32;
           if (!row_ok || n0 >= p.N) continue;
@@ -411,6 +461,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    // every TMA store of this warp has landed before the CTA goes away
+    if (!OUT_F32 && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   // neither CTA leaves (or frees tensor memory) while the other may still
@@ -427,8 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------ host side
 
 template <int FMT, int OUT_F32>
-cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const Params& p, int tiles,
-                         cudaStream_t s) {
+cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc,
+                         const Params& p, int tiles, cudaStream_t s) {
   auto kern = gemm_pair_kernel<FMT, OUT_F32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -459,7 +512,7 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const Par
   }
   const int pairs = std::max(1, std::min(tiles, max_pairs[dev]));
   cfg.gridDim = dim3(2 * pairs);
-  e = cudaLaunchKernelEx(&cfg, kern, ma, mw, p);
+  e = cudaLaunchKernelEx(&cfg, kern, ma, mw, mc, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -467,9 +520,13 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const Par
 }  // namespace
 
 cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
-  CUtensorMap ma, mw;
+  CUtensorMap ma, mw, mc;
   if (!make_code_map(&ma, a.a_codes, a.M, a.K, HALF)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, a.w_codes, a.N, a.K, HALF)) return cudaErrorInvalidValue;
+  if (a.out_f32)
+    mc = ma;   // unused by the fp32 epilogue
+  else if (!make_bf16_out_map(&mc, a.C, a.M, a.N, a.ldc, 32))
+    return cudaErrorInvalidValue;
   Params p;
   p.a_scales = a.a_scales;
   p.w_scales = a.w_scales;
@@ -490,8 +547,10 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
   if (!p.watchdog) return cudaErrorInvalidSymbol;
   const int tiles = p.m_tiles * p.n_tiles;
   if (a.fmt == 0)
-    return a.out_f32 ? launch_typed<0, 1>(ma, mw, p, tiles, s) : launch_typed<0, 0>(ma, mw, p, tiles, s);
-  return a.out_f32 ? launch_typed<1, 1>(ma, mw, p, tiles, s) : launch_typed<1, 0>(ma, mw, p, tiles, s);
+    return a.out_f32 ? launch_typed<0, 1>(ma, mw, mc, p, tiles, s)
+                     : launch_typed<0, 0>(ma, mw, mc, p, tiles, s);
+  return a.out_f32 ? launch_typed<1, 1>(ma, mw, mc, p, tiles, s)
+                   : launch_typed<1, 0>(ma, mw, mc, p, tiles, s);
 }
 
 }  // namespace fp4

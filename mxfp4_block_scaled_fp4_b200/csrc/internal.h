@@ -62,6 +62,10 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s);
 // rows and columns read as zero codes.
 bool make_code_map(CUtensorMap* m, const uint8_t* base, long long rows, int K, int box_rows);
 
+// Tensor map of a bf16 output C [rows, cols] with row pitch ldc elements:
+// box of 64 columns (128 bytes) by box_rows rows, 128-byte swizzle.
+bool make_bf16_out_map(CUtensorMap* m, void* C, long long rows, int cols, int ldc, int box_rows);
+
 struct FusedArgs {
   const void* a;        // bf16 [M, K]
   const uint8_t* w_codes; const uint8_t* w_scales; const float* g_w;
