@@ -42,7 +42,7 @@ FP4_OVER_BF16 = 4.0     # nominal dense FP4 / dense BF16 tensor throughput on B2
 # takes (gemm_pair_kernel), measured with ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass).  None whenever that kernel has changed
 # since it was last measured.
-GEMM_TRAFFIC_BYTES = None
+GEMM_TRAFFIC_BYTES = 307.2e6 + 435.5e6
 
 
 def load_peaks():
@@ -207,6 +207,54 @@ def measure_decode(torch, ops, L, inputs, dev, hbm_peak, shapes=None):
                     "weight_copies": copies})
         del graph, wqs
     return out
+
+
+def measure_vendor(torch, ops, inputs, dev, M, N, K):
+    """Context only: the vendor library's block-scaled FP4 GEMM (cuBLASLt,
+    reached through torch's scaled_mm) on the same quantized operands, bf16
+    out, timed like fp4_gemm (L2 flushed before each call).  Not part of the
+    product path; reports why if the library call is unavailable."""
+    try:
+        import torch.nn.functional as F
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        flush_r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        a, w = inputs.prefill(M, N, K)
+        res = {}
+        for fmt, name, sdt, rec in ((0, "nvfp4", torch.float8_e4m3fn, F.ScalingType.BlockWise1x16),
+                                    (1, "mxfp4", torch.float8_e8m0fnu, F.ScalingType.BlockWise1x32)):
+            aq = ops.quantize(a.to(dev), fmt, ops.SCALES_MMA)
+            wq = ops.quantize_weights(w.to(dev), fmt)
+            A = aq.codes.view(torch.float4_e2m1fn_x2)
+            B = wq.codes.view(torch.float4_e2m1fn_x2).t()
+            sa, sb = aq.scales.view(sdt), wq.scales.view(sdt)
+            sw = F.SwizzleType.SWIZZLE_32_4_4
+            c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            calls = {"ours": lambda: ops.gemm(aq, wq, out=c),
+                     "vendor": lambda: F.scaled_mm(A, B, sa, rec, sb, rec, sw, sw,
+                                                   output_dtype=torch.bfloat16)}
+            ms = {}
+            for key, fn in calls.items():
+                for _ in range(3):
+                    fn()
+                ts = []
+                for _ in range(10):
+                    flush_l2(torch, flush, flush_r)
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    fn()
+                    e1.record()
+                    torch.cuda.synchronize(dev)
+                    ts.append(e0.elapsed_time(e1))
+                ms[key] = float(np.median(ts))
+            fl = 2.0 * M * N * K
+            res[name] = {"ours_tflops": round(fl / ms["ours"] / 1e9, 1),
+                         "vendor_tflops": round(fl / ms["vendor"] / 1e9, 1),
+                         "ours_over_vendor": round(ms["vendor"] / ms["ours"], 3)}
+        res["vendor"] = "cuBLASLt block-scaled FP4 GEMM via torch.nn.functional.scaled_mm"
+        return res
+    except Exception as e:  # context only: never fails the bench
+        return {"unavailable": f"{type(e).__name__}: {str(e)[:200]}"}
 
 
 def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak):
@@ -478,7 +526,9 @@ def main():
         "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "format": "NVFP4",
                    "global_scale": "dynamic", "out": "bf16",
                    "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (A 128 MiB, packed W 131 MiB, C 448 MiB)"},
+                   "l2": (f"{'inputs larger than L2' if M * K * 2 > L2_BYTES else 'A fits in L2'} "
+                          f"(A {M * K * 2 >> 20} MiB, packed W {N * K // 2 >> 20} MiB, "
+                          f"C {M * N * 2 >> 20} MiB)")},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
                      "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
                      "traffic": GEMM_TRAFFIC_BYTES if (M, N, K) == (8192, 28672, 8192) else None,
@@ -500,6 +550,7 @@ def main():
         line["decode"] = measure_decode(torch, ops, L, inputs, dev, peaks["hbm_gbs"])
         line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"])
         line["decoder"] = measure_decoder(torch, dev)
+        line["vendor_reference"] = measure_vendor(torch, ops, inputs, dev, M, N, K)
         line["gpu_launches_note"] = ("gpu_launches counts the timed prefill steps only; the "
                                      "decode and sweep objects are timed separately")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
