@@ -228,11 +228,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Lean loop: the pipe runs one 256 x 256 x 64 MMA per 128 cycles and an
     // issue costs this thread ~75, so everything else it does between two
     // K steps must fit in ~200 cycles or the pipe idles (measured on B200).
-    // Descriptors advance by adding to their address field; the next
-    // stage's `ready` is polled while this stage's MMAs are queued.
+    // Descriptors advance by adding to their address field.  No extra
+    // probes of `ready`: an mbarrier.try_wait without a suspend hint that
+    // finds the phase incomplete can hold the thread for a system-defined
+    // time, which measured as a 25% slower K step.
     const uint64_t a_desc0 = smem_desc(smem_u32(sA), 16, 1024, kLayoutSwizzle128B);
     const uint64_t b_desc0 = smem_desc(smem_u32(sB), 16, 1024, kLayoutSwizzle128B);
-    const uint32_t ready0 = smem_u32(ready);
     const uint32_t sf0 = tmem + SF_COL;
     constexpr uint32_t kIdesc0 = idesc_fp4(BM, BN, FMT == 1, 0, 0);
     constexpr uint32_t kIdesc2 = idesc_fp4(BM, BN, FMT == 1, 2, 2);
@@ -241,7 +242,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
-    bool next_ready = false;
     for (int t = first; t < n_tiles_total; t += stride, ++it) {
       if (it > 0 && !mbar_wait(acc_empty, static_cast<uint32_t>(it - 1) & 1u, abort_flag,
                                p.watchdog, WD_MMA_ACC)) {
@@ -250,8 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       for (int kb = 0; kb < p.k_steps; ++kb) {
-        if (!next_ready && !mbar_try_wait(ready0 + stage * 8, phase) &&
-            !mbar_wait(&ready[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) {
+        if (!mbar_wait(&ready[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL)) {
           st_cluster_u32(peer_abort, 1u);
           goto mma_drain;
         }
@@ -263,7 +262,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           nphase ^= 1u;
         }
         const bool has_next = kb + 1 < p.k_steps;
-        next_ready = false;
         {
           const int n_mma = has_next ? BK / MMA_K : last_mmas;
           const uint64_t ad = a_desc0 + static_cast<uint64_t>(stage * (A_STAGE >> 4));
@@ -283,7 +281,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  (k & 1) ? kIdesc2 : kIdesc0, sfa_t + 4 * (k >> 1),
                                  sfb_t + 8 * (k >> 1), acc);
             }
-            if (k == 1 && has_next) next_ready = mbar_try_wait(ready0 + nstage * 8, nphase);
           }
         }
         tc_commit_pair(&empty[stage], 0x3);

@@ -51,20 +51,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-  return ok != 0;
-}
-
-// Same test, but a thread whose phase is not complete yet may be suspended
-// (up to kWaitSuspendNs) until it completes, instead of returning at once.
-// Waiting roles use this so that they do not take issue slots from the
-// warps that do work; measured on B200 it made the pair GEMM 7-8% faster.
+// Test whether phase `parity` of the barrier at shared address `bar` has
+// completed; if not, the thread may be suspended (up to kWaitSuspendNs)
+// until it completes.  (Without a hint the hardware picks the suspension
+// limit itself, so even an "unhinted" test is not a cheap probe.)  Waiting
+// roles suspending this way leave issue slots to the warps that do work;
+// measured on B200 that made the pair GEMM 7-8% faster.
 constexpr uint32_t kWaitSuspendNs = 100000u;
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
   uint32_t ok;
