@@ -18,11 +18,12 @@
 // 64 step); measured on B200 it is 8-13% faster than the one-CTA kernel on
 // large prefill shapes and bit-identical to it.
 //
-// Roles (10 warps in each CTA of the pair):
+// Roles (11 warps in each CTA of the pair):
 //   warp 0      TMA for this CTA: its A and W halves (plain, non-multicast
-//               tiled loads onto its own `full` barrier) and its scale atoms
-//               (the A row block of its half; both W row blocks of the tile,
-//               which every SM's MMA reads from its own tensor memory);
+//               tiled loads onto its own `full` barrier);
+//   warp 10     bulk copies of this CTA's scale atoms (the A row block of its
+//               half; both W row blocks of the tile, which every SM's MMA
+//               reads from its own tensor memory) onto `sf_loaded`;
 //   warp 1      both CTAs: tensor-memory allocation for the pair; leader,
 //               one thread: issues the pair MMAs, commits to both CTAs'
 //               `empty` / `acc_full` barriers (multicast commit);
@@ -74,7 +75,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = 256;
 constexpr uint32_t SF_STAGE_COLS = 48;
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;       // 11 warps
 constexpr int GROUP_M = 16;             // raster: 16 tile rows (4096 rows of A) share W in L2
 
 static_assert(SF_COL + STAGES * SF_STAGE_COLS <= TMEM_COLS, "scale stages exceed tensor memory");
@@ -177,30 +178,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = first; t < n_tiles_total; t += stride) {
       int mt, nt;
       tile_coords(t, p, mt, nt);
-      const int rba = mt * 2 + static_cast<int>(rank);   // A row block of this CTA's half
-      const bool a_rows = rba < p.a_rowblocks;
-      const int rb0 = nt * 2;
-      const int wblocks = min(2, p.w_rowblocks - rb0);
       for (int kb = 0; kb < p.k_steps; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.watchdog, WD_PRODUCER)) {
           st_cluster_u32(peer_abort, 1u);
           goto producer_drain;
         }
         {
-          const int cb0 = kb * kAtomsPerStage;
-          const int atoms = min(kAtomsPerStage, p.ncb - cb0);
-          const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
-          // a half made only of rows past M has no scale atoms; its
-          // accumulator rows are never stored
-          mbar_expect_tx(&sf_loaded[stage], sf_bytes * ((a_rows ? 1 : 0) + wblocks));
-          if (a_rows)
-            bulk_load(sSFA + stage * SFA_STAGE,
-                      p.a_scales + (static_cast<long long>(rba) * p.ncb + cb0) * 512, sf_bytes,
-                      &sf_loaded[stage]);
-          for (int i = 0; i < wblocks; ++i)
-            bulk_load(sSFB + stage * SFB_STAGE + i * 2048,
-                      p.w_scales + (static_cast<long long>(rb0 + i) * p.ncb + cb0) * 512, sf_bytes,
-                      &sf_loaded[stage]);
           mbar_expect_tx(&full[stage], A_STAGE + B_STAGE);
           tma_load_2d(sA + stage * A_STAGE, &tm_a, kb * BK_BYTES, mt * BM + rank * HALF,
                       &full[stage]);
@@ -218,11 +201,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     goto producer_done;
   producer_drain:
     for (int s = 0; s < STAGES; ++s)
-      if (armed & (1u << s)) {
-        mbar_wait_drain(&sf_loaded[s], (armed_parity >> s) & 1u, p.watchdog);
-        mbar_wait_drain(&full[s], (armed_parity >> s) & 1u, p.watchdog);
-      }
+      if (armed & (1u << s)) mbar_wait_drain(&full[s], (armed_parity >> s) & 1u, p.watchdog);
   producer_done:;
+  } else if (warp == 10 && lane == 0) {
+    // ------------------------------------------------ scale-atom producer
+    // A thread of its own, so that the scale copies and the code-tile
+    // copies of a stage are issued in parallel (each copy instruction costs
+    // its thread ~80 cycles, and this sits on the refill path of every stage)
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0, armed_parity = 0;
+    for (int t = first; t < n_tiles_total; t += stride) {
+      int mt, nt;
+      tile_coords(t, p, mt, nt);
+      const int rba = mt * 2 + static_cast<int>(rank);   // A row block of this CTA's half
+      const bool a_rows = rba < p.a_rowblocks;
+      const int rb0 = nt * 2;
+      const int wblocks = min(2, p.w_rowblocks - rb0);
+      const uint8_t* sfa_g = p.a_scales + static_cast<long long>(rba) * p.ncb * 512;
+      const uint8_t* sfb_g = p.w_scales + static_cast<long long>(rb0) * p.ncb * 512;
+      for (int kb = 0; kb < p.k_steps; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.watchdog, WD_PRODUCER)) {
+          st_cluster_u32(peer_abort, 1u);
+          goto sf_drain;
+        }
+        {
+          const int cb0 = kb * kAtomsPerStage;
+          const int atoms = min(kAtomsPerStage, p.ncb - cb0);
+          const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
+          // a half made only of rows past M has no scale atoms; its
+          // accumulator rows are never stored
+          mbar_expect_tx(&sf_loaded[stage], sf_bytes * ((a_rows ? 1 : 0) + wblocks));
+          if (a_rows)
+            bulk_load(sSFA + stage * SFA_STAGE, sfa_g + cb0 * 512, sf_bytes, &sf_loaded[stage]);
+          for (int i = 0; i < wblocks; ++i)
+            bulk_load(sSFB + stage * SFB_STAGE + i * 2048,
+                      sfb_g + (static_cast<long long>(i) * p.ncb + cb0) * 512, sf_bytes,
+                      &sf_loaded[stage]);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    goto sf_done;
+  sf_drain:
+    for (int s = 0; s < STAGES; ++s)
+      if (armed & (1u << s)) mbar_wait_drain(&sf_loaded[s], (armed_parity >> s) & 1u, p.watchdog);
+  sf_done:;
   } else if (warp == 1 && lane == 0 && leader) {
     // ---------------------------------------------------- pair MMA issuer
     // Lean loop: the pipe runs one 256 x 256 x 64 MMA per 128 cycles and an
@@ -294,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_commit_pair(drain, 0x1);
     mbar_wait_drain(drain, 0, p.watchdog);
   mma_done:;
-  } else if (warp >= 6) {
+  } else if (warp >= 6 && warp <= 9) {
     // ----------------------------------------------------- scale staging
     const int quarter = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -355,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   staging_done:;
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     float alpha = 1.0f;
