@@ -1,12 +1,11 @@
-// codec.cuh -- device-side NVFP4 / MXFP4 element and scale codecs, shared by
-// the stand-alone quantizer (quantize.cu) and the fused small-M kernel
-// (fused.cu), so both produce identical codes.
+// codec.cuh -- device-side NVFP4 / MXFP4 element and scale codecs of the
+// quantizer (quantize.cu).
 //
 // "Hardware FP4 inference for speech on Blackwell", section "NVFP4, and the
 // two ways it fails": E2M1 code points {0, 0.5, 1, 1.5, 2, 3, 4, 6}, E4M3
 // block scale with maximum 448.  MXFP4 E8M0 scale: "FP4 n'existe pas", format
-// table.  Every floating-point step is one explicitly rounded binary32
-// operation (no contraction).
+// table.  Every floating-point step yields the correctly rounded binary32
+// result of that step (explicitly rounded operations, no contraction).
 #pragma once
 #include <cstdint>
 
@@ -16,15 +15,19 @@ namespace fp4 {
 // finite values the 15-bit pattern orders like the magnitude.
 __device__ __forceinline__ unsigned bf16x2_mag(unsigned w) { return w & 0x7FFF7FFFu; }
 
+// Lane-wise maximum of two pairs of 16-bit unsigned values (native on sm_90+).
+__device__ __forceinline__ unsigned max_u16x2(unsigned a, unsigned b) {
+  unsigned d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 __device__ __forceinline__ unsigned mag_max8(uint4 v) {
-  return __vmaxu2(__vmaxu2(bf16x2_mag(v.x), bf16x2_mag(v.y)),
-                  __vmaxu2(bf16x2_mag(v.z), bf16x2_mag(v.w)));
+  return max_u16x2(max_u16x2(bf16x2_mag(v.x), bf16x2_mag(v.y)),
+                   max_u16x2(bf16x2_mag(v.z), bf16x2_mag(v.w)));
 }
 
 __device__ __forceinline__ unsigned fold_u16x2(unsigned m) { return max(m & 0xFFFFu, m >> 16); }
-
-__device__ __forceinline__ float bf16_lo(unsigned w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(unsigned w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // E4M3 (round to nearest even, saturating at 448) of a non-negative float.
 __device__ __forceinline__ unsigned to_e4m3(float v) {
@@ -40,38 +43,51 @@ __device__ __forceinline__ float e4m3_value(unsigned c) {
   return __uint_as_float(((e + 120u) << 23) | (m << 20));         // (8+m) 2^(e-10)
 }
 
-// Eight floats -> eight E2M1 nibbles (value i in nibble i), round to
-// nearest even, saturating at 6.
-__device__ __forceinline__ unsigned to_e2m1x8(float v0, float v1, float v2, float v3, float v4,
-                                              float v5, float v6, float v7) {
+// 8 bf16 (4 words, element 2i in the low half of word i) times r -> 8
+// packed E2M1 codes (element i in nibble i).  Each product is one binary32
+// multiply rounded to nearest (two per mul.rn.f32x2, measured on B200 to be
+// bit-identical to two scalar multiplies), then round to nearest even,
+// saturating at 6.  The conversion keeps the sign of a negative product that
+// rounds to zero (code 0x8), measured on B200 for every such input tried,
+// -0.0 included; that is the sign rule of the format.
+__device__ __forceinline__ unsigned quant8(unsigned w0, unsigned w1, unsigned w2, unsigned w3,
+                                           float r) {
   unsigned out;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+  asm("{\n\t"
+      ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+      ".reg .b64 x0, x1, x2, x3, rr;\n\t"
+      ".reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b64 rr, {%5, %5};\n\t"
+      "shl.b32 l0, %1, 16;\n\t and.b32 h0, %1, 0xFFFF0000;\n\t mov.b64 x0, {l0, h0};\n\t"
+      "shl.b32 l1, %2, 16;\n\t and.b32 h1, %2, 0xFFFF0000;\n\t mov.b64 x1, {l1, h1};\n\t"
+      "shl.b32 l2, %3, 16;\n\t and.b32 h2, %3, 0xFFFF0000;\n\t mov.b64 x2, {l2, h2};\n\t"
+      "shl.b32 l3, %4, 16;\n\t and.b32 h3, %4, 0xFFFF0000;\n\t mov.b64 x3, {l3, h3};\n\t"
+      "mul.rn.f32x2 x0, x0, rr;\n\t mul.rn.f32x2 x1, x1, rr;\n\t"
+      "mul.rn.f32x2 x2, x2, rr;\n\t mul.rn.f32x2 x3, x3, rr;\n\t"
+      "mov.b64 {l0, h0}, x0;\n\t mov.b64 {l1, h1}, x1;\n\t"
+      "mov.b64 {l2, h2}, x2;\n\t mov.b64 {l3, h3}, x3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, h0, l0;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, h1, l1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, h2, l2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, h3, l3;\n\t"
       "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
       : "=r"(out)
-      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+      : "r"(w0), "r"(w1), "r"(w2), "r"(w3), "f"(r));
   return out;
 }
 
-// Sign bits of four bf16x2 words moved to bit 3 of each nibble: the code of
-// a negative input carries its sign, also when it rounds to zero.
-__device__ __forceinline__ unsigned sign_nibbles(unsigned w0, unsigned w1, unsigned w2,
-                                                 unsigned w3) {
-  auto s = [](unsigned w) { return ((w >> 12) & 0x8u) | ((w >> 24) & 0x80u); };
-  return s(w0) | s(w1) << 8 | s(w2) << 16 | s(w3) << 24;
-}
-
-// 8 bf16 (4 words) times r -> 8 packed E2M1 codes.
-__device__ __forceinline__ unsigned quant8(unsigned w0, unsigned w1, unsigned w2, unsigned w3,
-                                           float r) {
-  const unsigned q = to_e2m1x8(__fmul_rn(bf16_lo(w0), r), __fmul_rn(bf16_hi(w0), r),
-                               __fmul_rn(bf16_lo(w1), r), __fmul_rn(bf16_hi(w1), r),
-                               __fmul_rn(bf16_lo(w2), r), __fmul_rn(bf16_hi(w2), r),
-                               __fmul_rn(bf16_lo(w3), r), __fmul_rn(bf16_hi(w3), r));
-  return q | sign_nibbles(w0, w1, w2, w3);
+// RN(a / b) for a >= 0 by Markstein's method (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", 1990): with
+// y = RN(1/b) and q1 = RN(a y), the remainder a - b q1 is exact in one FMA
+// and RN(q1 + (a - b q1) y) is the correctly rounded quotient, provided no
+// intermediate under- or overflows.  fast_b says b lies in [2^-40, 2^40];
+// with q1 also in that range every intermediate is a normal number, outside
+// it the division itself runs.  Checked on B200 against the correctly
+// rounded division for every positive finite bf16 a and 4000 divisors.
+__device__ __forceinline__ float div_rn(float a, float b, float y, bool fast_b) {
+  const float q1 = __fmul_rn(a, y);
+  if (fast_b && q1 >= 0x1p-40f && q1 <= 0x1p40f) return __fmaf_rn(__fmaf_rn(-q1, b, a), y, q1);
+  return __fdiv_rn(a, b);
 }
 
 // floor(log2(b)) of a positive finite float, from its bits.
@@ -82,14 +98,19 @@ __device__ __forceinline__ int floor_log2(float b) {
   return (31 - __clz(u & 0x7FFFFFu)) - 149;
 }
 
-// One 16-value NVFP4 block: magnitude bits of its max -> E4M3 scale byte and
-// the reciprocal r = 1 / (s g) (0 when the scale rounds to zero).
-__device__ __forceinline__ unsigned nvfp4_scale(unsigned amax_bits, float g, float six_g,
-                                                float* r) {
-  const unsigned s = to_e4m3(__fdiv_rn(__uint_as_float(amax_bits << 16), six_g));
+// One 16-value NVFP4 block: magnitude bits of its max -> E4M3 scale byte
+// s = E4M3(RN(amax / RN(6 g))).  (y6 = RN(1 / RN(6 g)).)
+__device__ __forceinline__ unsigned nvfp4_scale_byte(unsigned amax_bits, float six_g, float y6,
+                                                     bool fast_b) {
+  return to_e4m3(div_rn(__uint_as_float(amax_bits << 16), six_g, y6, fast_b));
+}
+
+// The reciprocal the block's values are multiplied by: r = RN(1 / RN(s g)),
+// 0 when the scale is zero.  It depends on the scale byte alone, so the
+// quantizer tabulates it per CTA.
+__device__ __forceinline__ float nvfp4_recip(unsigned s, float g) {
   const float sv = e4m3_value(s);
-  *r = (sv == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sv, g));
-  return s;
+  return (sv == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sv, g));
 }
 
 // One 32-value MXFP4 block: E8M0 scale byte and r = 2^-e.

@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const uint4* __restri
       v[j] = (i < n_vec) ? ld_stream(x + i) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) m = __vmaxu2(m, mag_max8(v[j]));
+    for (int j = 0; j < 4; ++j) m = max_u16x2(m, mag_max8(v[j]));
   }
   m = fold_u16x2(m);
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -99,19 +99,41 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const uint4* __restri
 
 // -------------------------------------------------------- quantize pass
 
+// n / d for 32-bit n by multiply-high (Granlund & Montgomery, "Division by
+// invariant integers using multiplication", 1994): l = ceil(log2 d),
+// m = floor(2^32 (2^l - d) / d) + 1, q = (mulhi(n, m) + n) >> l; d = 1 is
+// m = 0, l = 0.
+struct FastDiv {
+  unsigned m;
+  unsigned l;
+};
+__device__ __forceinline__ unsigned fast_div(unsigned n, FastDiv f) {
+  return static_cast<unsigned>((static_cast<unsigned long long>(__umulhi(n, f.m)) + n) >> f.l);
+}
+
 // A warp quantizes a slab of 4 x 32 consecutive units per iteration: every
 // lane issues its 8 loads (4 units x 32 bytes) before computing.  With a
 // DYNAMIC global scale the slabs are walked from the end, so the first ones
 // are still in L2 from the amax pass.
 template <int FMT, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long long units,
-                                                               int upr, int nsf, int ncb,
-                                                               long long pad_a, long long pad_b) {
+                                                               int upr, FastDiv upr_div, int nsf,
+                                                               int ncb, long long pad_a,
+                                                               long long pad_b) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float g = (FMT == 0) ? global_scale(a.dynamic, a.g, a.partial, a.n_partial) : 1.0f;
   if (FMT == 0 && a.dynamic && blockIdx.x == 0 && threadIdx.x == 0) *a.g = g;
   const float six_g = __fmul_rn(6.0f, g);
+  const float y6 = __frcp_rn(six_g);
+  const bool fast_b = six_g >= 0x1p-40f && six_g <= 0x1p40f;
+  // r = RN(1 / RN(s g)) for every scale byte this pass can produce (s <= 0x7F)
+  __shared__ float r_tab[128];
+  if (FMT == 0) {
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) r_tab[i] = nvfp4_recip(i, g);
+    __syncthreads();
+  }
+  const bool big = units > 0xFFFFFFFFll;   // unit indices beyond 32 bits: plain division
 
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
   uint2* __restrict__ codes = reinterpret_cast<uint2*>(a.codes);
@@ -139,12 +161,13 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long
     for (int j = 0; j < 4; ++j) {
       const long long u = slab * 128 + j * 32 + lane;
       const uint4 p = xs[j][0], q = xs[j][1];
-      unsigned m = fold_u16x2(__vmaxu2(mag_max8(p), mag_max8(q)));
+      unsigned m = fold_u16x2(max_u16x2(mag_max8(p), mag_max8(q)));
       unsigned sbyte;
       uint2 packed;
       float r;
       if (FMT == 0) {
-        sbyte = nvfp4_scale(m, g, six_g, &r);
+        sbyte = nvfp4_scale_byte(m, six_g, y6, fast_b);
+        r = r_tab[sbyte & 127u];
         packed = (r == 0.0f) ? make_uint2(0, 0)
                              : make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
       } else {
@@ -154,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long
       }
       if (u < units) {
         codes[u] = packed;
-        const long long row = u / upr;
+        const long long row =
+            big ? u / upr : static_cast<long long>(fast_div(static_cast<unsigned>(u), upr_div));
         const int jj = static_cast<int>(u - row * upr);
         if (FMT == 0 || (jj & 1) == 0) {
           const int c = (FMT == 0) ? jj : (jj >> 1);
@@ -246,7 +270,15 @@ cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl) {
       std::max<long long>(1, std::min<long long>(want, static_cast<long long>(sm_count()) * 4)));
   auto kern = (a.fmt == 0) ? (a.layout == 0 ? quantize_kernel<0, 0> : quantize_kernel<0, 1>)
                            : (a.layout == 0 ? quantize_kernel<1, 0> : quantize_kernel<1, 1>);
-  const cudaError_t e = launch_k(kern, blocks, pdl, s, a, units, upr, nsf, ncb, pad_a, pad_b);
+  FastDiv fd{0u, 0u};
+  if (upr > 1) {
+    unsigned l = 0;
+    while ((1ull << l) < static_cast<unsigned long long>(upr)) ++l;
+    fd.l = l;
+    fd.m = static_cast<unsigned>(((1ull << 32) * ((1ull << l) - static_cast<unsigned long long>(upr))) /
+                                     static_cast<unsigned long long>(upr) + 1);
+  }
+  const cudaError_t e = launch_k(kern, blocks, pdl, s, a, units, upr, fd, nsf, ncb, pad_a, pad_b);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
