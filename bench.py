@@ -42,7 +42,7 @@ FP4_OVER_BF16 = 4.0     # nominal dense FP4 / dense BF16 tensor throughput on B2
 # takes (gemm_pair_kernel), measured with ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass).  None whenever that kernel has changed
 # since it was last measured.
-GEMM_TRAFFIC_BYTES = 307.2e6 + 435.5e6
+GEMM_TRAFFIC_BYTES = 306.7e6 + 435.2e6
 
 
 def load_peaks():

@@ -95,6 +95,27 @@ def test_crafted_edge_blocks(ops, orc, fmt, g):
     check_quant(ops, orc, crafted(), fmt, g)
 
 
+def ladder(top=50):
+    """One 16-value block per power of two from 2^-70 to 2^top (mantissas
+    drawn at random, signs mixed), so the block maxima straddle both ends of
+    the range in which the quantizer computes amax / (6 g) by Markstein's
+    method rather than by a division."""
+    g = np.random.default_rng(11)
+    exps = np.arange(-70, top + 1)
+    blocks = (g.uniform(1.0, 2.0, size=(exps.size, 16)) * np.exp2(exps)[:, None]
+              * np.where(g.random((exps.size, 16)) < 0.5, -1.0, 1.0))
+    flat = blocks.astype(np.float32).reshape(-1)
+    K = 256
+    flat = np.concatenate([flat, np.zeros((-flat.size) % K, np.float32)])
+    return inputs.to_bf16(flat.reshape(-1, K))
+
+
+@pytest.mark.parametrize("top", [50, 10])
+@pytest.mark.parametrize("g", [None, 1e-20, 3.0e-4, 1.0, 1e20])
+def test_scale_division_paths(ops, orc, top, g):
+    check_quant(ops, orc, ladder(top), 0, g_static=g)
+
+
 def test_zero_rows_is_a_noop(ops):
     x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
     q = ops.quantize(x, 0, ops.SCALES_MMA)
