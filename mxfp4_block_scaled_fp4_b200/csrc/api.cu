@@ -137,7 +137,10 @@ fp4_status_t fp4_quantize_act(const void* x, int rows, int K, fp4_format_t fmt,
     a.partial = partial;
     a.n_partial = used;
   }
-  return from_cuda(fp4::launch_quantize(a, s));
+  // DYNAMIC: the quantize pass is a programmatic dependent of the amax pass
+  // (it waits for the amax grid before reading), so its launch overlaps the
+  // amax pass's tail
+  return from_cuda(fp4::launch_quantize(a, s, dyn));
 }
 
 fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt, uint8_t* codes,
