@@ -444,6 +444,8 @@ cudaError_t launch_gemm_fused(const FusedArgs& f, cudaStream_t s) {
   // and 0 x NaN would not be 0); rows >= M only reach output columns that
   // are never stored
   q.zero_pad_rows = 0;
+  // the GEMM reads the quantized activation only after its wait
+  q.release_early = 1;
   cudaError_t e;
   if (f.dynamic) {
     int used = 0;

@@ -44,6 +44,12 @@ struct QuantArgs {
   // MMA layout: also zero the scales of rows [rows, rows rounded up to 128).
   // The small-M GEMM never reads those rows' scales, so its chain skips it.
   int zero_pad_rows = 1;
+  // Release the next kernel of the stream at once (programmatic dependent
+  // launch) instead of at completion.  Only for a dependent known to read
+  // this pass's output after its griddepcontrol.wait: the small-M GEMM may
+  // stream its weights before that wait, so a pass that could be writing
+  // weights must never release it early.
+  int release_early = 0;
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl = false);
 

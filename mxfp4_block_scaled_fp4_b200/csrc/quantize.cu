@@ -65,9 +65,11 @@ __device__ float global_scale(int dynamic, const float* g, const unsigned* parti
 __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const uint4* __restrict__ x,
                                                            long long n_vec,
                                                            unsigned* __restrict__ partial) {
-  // In a programmatic-dependent-launch chain (the small-M path) the next
-  // kernel may launch now; the input is read only after the previous
-  // kernel finished.  Without such a launch both are no-ops.
+  // In a programmatic-dependent-launch chain the next kernel may launch now
+  // (this pass writes nothing but its own partial maxima, which only the
+  // quantize pass reads, after its griddepcontrol.wait); the input is read
+  // only after the previous kernel finished.  Without such a launch both are
+  // no-ops.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long
                                                                int upr, FastDiv upr_div, int nsf,
                                                                int ncb, long long pad_a,
                                                                long long pad_b) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (a.release_early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float g = (FMT == 0) ? global_scale(a.dynamic, a.g, a.partial, a.n_partial) : 1.0f;
   if (FMT == 0 && a.dynamic && blockIdx.x == 0 && threadIdx.x == 0) *a.g = g;
