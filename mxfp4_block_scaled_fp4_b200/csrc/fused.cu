@@ -118,7 +118,7 @@ __device__ __forceinline__ float ld_peer_f32(uint32_t local_saddr, uint32_t rank
   uint32_t remote;
   float v;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote));
   return v;
 }
 
@@ -366,10 +366,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const int n = tile * FBM + t;
       const uint32_t base = smem_u32(sW) + t * 4;
       // CTA `split` reduces rows m = split, split + S, ... in slice order
+      // all S remote loads of a row are issued before the first add
       for (int m = split; m < p.M; m += p.splits) {
+        float v[kMaxSplits];
+#pragma unroll
+        for (int s = 0; s < kMaxSplits; ++s)
+          v[s] = (s < p.splits) ? ld_peer_f32(base + m * FBM * 4, static_cast<uint32_t>(s)) : 0.0f;
         float acc = 0.0f;
-        for (int s = 0; s < p.splits; ++s)
-          acc = __fadd_rn(acc, ld_peer_f32(base + m * FBM * 4, static_cast<uint32_t>(s)));
+#pragma unroll
+        for (int s = 0; s < kMaxSplits; ++s)
+          if (s < p.splits) acc = __fadd_rn(acc, v[s]);
         if (n < p.N) store_out(p, m, n, __fmul_rn(alpha, acc));
       }
     }
@@ -424,6 +430,7 @@ size_t fused_workspace_bytes(int M, int N, int K, int fmt) {
 }
 
 cudaError_t launch_gemm_fused(const FusedArgs& f, cudaStream_t s) {
+  if (decode_supported(f.M, f.N, f.K)) return launch_decode(f, s);
   const Plan pl = make_plan(f.M, f.N, f.K, f.fmt);
   uint8_t* ws = static_cast<uint8_t*>(f.ws);
   uint8_t* x_codes = ws + pl.off_codes;

@@ -84,5 +84,9 @@ size_t fused_workspace_bytes(int M, int N, int K, int fmt);
 // Shapes the fused path takes: 1 <= M <= 32 and K up to 8 slices of 8192.
 bool fused_supported(int M, int N, int K);
 cudaError_t launch_gemm_fused(const FusedArgs& a, cudaStream_t s);
+// The one-kernel path of launch_gemm_fused (M <= 32, M * K <= 128K values,
+// K slices of at most 8 steps of 256).
+bool decode_supported(int M, int N, int K);
+cudaError_t launch_decode(const FusedArgs& a, cudaStream_t s);
 
 }  // namespace fp4

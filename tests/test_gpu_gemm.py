@@ -99,8 +99,10 @@ def test_prefill_full_size_sampled(ops, orc, M, N, K, fmt, dt):
     assert ok, f"worst err/bound {worst:.3g} at {where}"
 
 
+# M * K <= 128K values take the one-kernel path, larger activations the
+# amax -> quantize -> GEMM chain (the last two shapes)
 FUSED_RAGGED = [(1, 8, 32), (5, 264, 2880), (16, 520, 1056), (17, 136, 96), (32, 1024, 4096),
-                (32, 14336, 256), (3, 4096, 8192)]
+                (32, 14336, 256), (3, 4096, 8192), (24, 1032, 8192), (32, 520, 8192)]
 
 
 @pytest.mark.parametrize("M,N,K", FUSED_RAGGED)
