@@ -56,7 +56,11 @@ constexpr int DXS_STEP = kMaxRows * 16;         // activation scales per step, 1
 constexpr int kMaxSplits = 8;                // portable cluster size
 constexpr int kThreads = 192;
 constexpr int kTargetCtas = 2 * 148;         // one wave of two CTAs per SM
-constexpr long long kMaxActValues = 131072;  // 256 KiB of bf16 read by every CTA
+// Every CTA reads the whole activation (amax) and quantizes M x its K slice:
+// beyond these sizes the three-kernel chain, which quantizes once, is faster
+// (measured on B200).
+constexpr long long kMaxActValues = 32768;   // 64 KiB of bf16 read by every CTA
+constexpr int kMaxSliceValues = 16384;       // values quantized by one CTA
 constexpr int SMEM_BYTES =
     1024 + DSTAGES * (DW_STAGE + DSF_STAGE) + kMaxSteps * (DX_STEP + DXS_STEP) + 512 + 256;
 constexpr uint32_t D_TMEM_COLS = 256;
@@ -83,8 +87,9 @@ DPlan make_dplan(int M, int N, int K) {
   for (int t = 2; t <= kMaxSplits && t <= p.k_steps; ++t)
     if (p.n_tiles * t <= kTargetCtas) s = t;
   p.splits = s;
+  const int slice_steps = (p.k_steps + s - 1) / s;
   p.ok = M >= 1 && M <= kMaxRows && static_cast<long long>(M) * K <= kMaxActValues &&
-         (p.k_steps + s - 1) / s <= kMaxSteps;
+         slice_steps <= kMaxSteps && M * slice_steps * DBK <= kMaxSliceValues;
   return p;
 }
 
@@ -286,14 +291,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.dynamic) {
         unsigned m = 0;
         const long long n_vec = static_cast<long long>(p.M) * p.K / 8;
-        // four 16-byte loads in flight per thread
-        for (long long v = wt; v < n_vec; v += 512) {
-          uint4 t[4];
+        // eight 16-byte loads in flight per thread
+        for (long long v = wt; v < n_vec; v += 1024) {
+          uint4 t[8];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < 8; ++j)
             t[j] = (v + 128 * j < n_vec) ? ld_x16(p.x + (v + 128 * j) * 8) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) m = max_u16x2(m, mag_max8(t[j]));
+          for (int j = 0; j < 8; ++j) m = max_u16x2(m, mag_max8(t[j]));
         }
         m = fold_u16x2(m);
         for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -317,19 +322,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float six_g = __fmul_rn(6.0f, g);
       const float y6 = __frcp_rn(six_g);
       const bool fast_b = six_g >= 0x1p-40f && six_g <= 0x1p40f;
+      uint4 nx0 = pre0, nx1 = pre1;
       for (int base = 0; base < units; base += 128) {
         const int u = base + wt;
         const bool valid = u < units;
         const int m = valid ? u / upr : 0;
         const int i = valid ? u - m * upr : 0;
-        uint4 a0 = pre0, a1 = pre1;
-        if (base > 0) {
-          a0 = a1 = make_uint4(0u, 0u, 0u, 0u);
-          if (valid) {
-            const uint16_t* src = p.x + static_cast<long long>(m) * p.K + k0 + 16 * i;
-            a0 = ld_x16(src);
-            a1 = ld_x16(src + 8);
-          }
+        const uint4 a0 = nx0, a1 = nx1;
+        // the next batch's loads go out before this batch is converted
+        nx0 = nx1 = make_uint4(0u, 0u, 0u, 0u);
+        if (u + 128 < units) {
+          const int mn = (u + 128) / upr, in = u + 128 - mn * upr;
+          const uint16_t* src = p.x + static_cast<long long>(mn) * p.K + k0 + 16 * in;
+          nx0 = ld_x16(src);
+          nx1 = ld_x16(src + 8);
         }
         unsigned mx = fold_u16x2(max_u16x2(mag_max8(a0), mag_max8(a1)));
         unsigned sbyte;
