@@ -173,6 +173,18 @@ fp4_status_t fp4_gemm_fused(const void* a, const uint8_t* w_codes, const uint8_t
  * the last call's contents; no clearing is needed since every call writes
  * each slot before reading it.  No cudaMalloc / cudaFree or other allocating
  * call is made. */
+/* The launch shape fp4_gemm takes for an M x N x K problem on the current
+ * device, for tests and profiling (nothing is launched; the pages have no
+ * counterpart).  *tile_m x *tile_n output tiles (256 x 256: the CTA-pair
+ * kernel; 128 x {256, 128, 64}: one CTA per tile) and *splits CTAs per tile
+ * along K: a thread-block cluster whose CTAs each accumulate one slice of K
+ * and then add their FP32 partial sums in a fixed order (split 0 first), so
+ * repeated calls give identical bits.  Narrow tiles and splits are taken
+ * when 256-wide tiles would leave most SMs idle.  Errors as fp4_gemm's
+ * shape checks, FP4_ERR_INVALID_ARG for a NULL output pointer. */
+fp4_status_t fp4_gemm_plan(int M, int N, int K, fp4_format_t fmt,
+                           int* tile_m, int* tile_n, int* splits);
+
 fp4_status_t fp4_quantize_act_noalloc(const void* x, int rows, int K, fp4_format_t fmt,
                                       fp4_scale_layout_t layout, fp4_global_mode_t gmode,
                                       float* g, uint8_t* codes, uint8_t* scales,

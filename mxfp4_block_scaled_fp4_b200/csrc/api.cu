@@ -132,15 +132,17 @@ fp4_status_t fp4_quantize_act(const void* x, int rows, int K, fp4_format_t fmt,
   if (dyn) {
     int used = 0;
     unsigned* partial = static_cast<unsigned*>(ws);
-    if (fp4::launch_amax(x, static_cast<long long>(rows) * K, partial, &used, s) != cudaSuccess)
+    if (fp4::launch_amax(x, static_cast<long long>(rows) * K, partial, &used, s, true) !=
+        cudaSuccess)
       return FP4_ERR_CUDA;
     a.partial = partial;
     a.n_partial = used;
   }
-  // DYNAMIC: the quantize pass is a programmatic dependent of the amax pass
-  // (it waits for the amax grid before reading), so its launch overlaps the
-  // amax pass's tail
-  return from_cuda(fp4::launch_quantize(a, s, dyn));
+  // Both passes are programmatic dependents of the kernel before them (each
+  // waits for its predecessor before reading), so their launches overlap
+  // the predecessor's tail.  The quantize pass does not release its own
+  // dependent early: a fused GEMM may read weights before its wait.
+  return from_cuda(fp4::launch_quantize(a, s, true));
 }
 
 fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt, uint8_t* codes,
@@ -187,6 +189,17 @@ fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const flo
   a.ldc = ldc;
   a.out_f32 = out == FP4_OUT_F32;
   return from_cuda(fp4::launch_gemm(a, static_cast<cudaStream_t>(stream)));
+}
+
+fp4_status_t fp4_gemm_plan(int M, int N, int K, fp4_format_t fmt, int* tile_m, int* tile_n,
+                           int* splits) {
+  fp4_status_t st;
+  if ((st = check_format(fmt)) != FP4_OK) return st;
+  if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!tile_m || !tile_n || !splits) return FP4_ERR_INVALID_ARG;
+  if ((st = device_ok()) != FP4_OK) return st;
+  return from_cuda(fp4::gemm_plan(M, N, K, tile_m, tile_n, splits));
 }
 
 fp4_status_t fp4_gemm_fused(const void* x, const uint8_t* w_codes, const uint8_t* w_scales,

@@ -60,7 +60,10 @@ struct GemmArgs {
   void* C; int ldc; int out_f32;
 };
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s);
-// The CTA-pair kernel (256-row tiles); launch_gemm takes it for M > 128.
+// The shape launch_gemm takes: tile rows x columns, CTAs per tile along K.
+cudaError_t gemm_plan(int M, int N, int K, int* tile_m, int* tile_n, int* splits);
+// The CTA-pair kernel (256 x 256 tiles); launch_gemm takes it for M > 128
+// when its tiles keep at least half the SMs busy.
 cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s);
 
 // Tensor map of packed FP4 codes [rows, K/2] bytes as a 2-D uint8 tensor:

@@ -60,6 +60,7 @@ SIGNATURES = {
     "fp4_quantize_weights": (I, [P, I, I, I, U8P, U8P, FP, P, SZ, P]),
     "fp4_gemm": (I, [U8P, U8P, FP, U8P, U8P, FP, I, I, I, I, P, I, I, P, SZ, P]),
     "fp4_gemm_fused": (I, [P, U8P, U8P, FP, I, I, I, I, I, FP, P, I, I, P, SZ, P]),
+    "fp4_gemm_plan": (I, [I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
     "fp4_quantize_act_noalloc": (I, [P, I, I, I, I, I, FP, U8P, U8P, P]),
     "fp4_device_status": (I, [ctypes.POINTER(ctypes.c_uint), P]),
     "fp4_watchdog_selftest": (I, [ctypes.c_ulonglong, P]),
@@ -127,6 +128,10 @@ def fp4_gemm_fused(a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc, 
                    ws_bytes, stream):
     return _call("fp4_gemm_fused", a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc,
                  out, ws, ws_bytes, stream)
+
+
+def fp4_gemm_plan(M, N, K, fmt, tile_m, tile_n, splits):
+    return _call("fp4_gemm_plan", M, N, K, fmt, tile_m, tile_n, splits)
 
 
 def fp4_quantize_act_noalloc(x, rows, K, fmt, layout, gmode, g, codes, scales, stream):

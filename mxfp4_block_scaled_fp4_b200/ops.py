@@ -8,6 +8,8 @@ from __future__ import annotations
 
 from dataclasses import dataclass
 
+import ctypes
+
 import torch
 
 from . import fp4lib as L
@@ -105,6 +107,14 @@ def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
                       w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(), M, N, K, a.fmt,
                       out.data_ptr(), out.stride(0), o, None, 0, _stream()), "fp4_gemm")
     return out
+
+
+def gemm_plan(M: int, N: int, K: int, fmt: int = NVFP4) -> tuple[int, int, int]:
+    """fp4_gemm_plan: (tile_m, tile_n, splits) that fp4_gemm launches."""
+    tm, tn, sp = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(L.fp4_gemm_plan(M, N, K, fmt, ctypes.byref(tm), ctypes.byref(tn), ctypes.byref(sp)),
+           "fp4_gemm_plan")
+    return tm.value, tn.value, sp.value
 
 
 def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,

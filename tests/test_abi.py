@@ -50,6 +50,15 @@ def test_scale_bytes_match_oracle_layout(lib, orc):
             orc.mma_scale_bytes(rows, K // 32)
 
 
+def test_gemm_plan_argument_checks(lib):
+    i = [ctypes.c_int() for _ in range(3)]
+    refs = [ctypes.byref(x) for x in i]
+    assert L.fp4_gemm_plan(8, 256, 100, 0, *refs) == L.FP4_ERR_UNSUPPORTED_SHAPE   # K % 32
+    assert L.fp4_gemm_plan(8, 260, 256, 0, *refs) == L.FP4_ERR_UNSUPPORTED_SHAPE   # N % 8
+    assert L.fp4_gemm_plan(8, 256, 256, 7, *refs) == L.FP4_ERR_INVALID_ARG
+    assert L.fp4_gemm_plan(8, 256, 256, 0, None, refs[1], refs[2]) == L.FP4_ERR_INVALID_ARG
+
+
 def test_argument_checks_fail_before_any_launch(lib):
     fake = ctypes.c_void_p(1 << 20)           # never dereferenced: checks fail first
     mis = ctypes.c_void_p((1 << 20) + 8)

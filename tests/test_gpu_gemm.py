@@ -52,7 +52,25 @@ def test_pr1_tiny_outliers(ops, orc, fmt, dt, fused):
 
 
 RAGGED = [(1, 8, 32), (16, 256, 64), (130, 264, 2880), (300, 520, 1056), (257, 512, 4096),
-          (128, 256, 256), (129, 136, 96), (2304, 2312, 320)]
+          (128, 256, 256), (129, 136, 96), (2304, 2312, 320), (600, 4104, 1056), (1024, 4096, 128),
+          # few output tiles: narrow tiles and / or K split across a cluster
+          (256, 2880, 2880), (64, 2880, 2880), (8, 720, 7680), (8, 256, 2048),
+          (200, 1024, 6400), (200, 4864, 256), (8, 19200, 256), (256, 2880, 7680)]
+
+
+# Launch classes fp4_gemm can take: (tile rows, tile columns, split along K);
+# K is split only with 64- and 128-wide tiles
+LAUNCH_CLASSES = {(256, 256, False), (128, 256, False), (128, 128, False), (128, 128, True),
+                  (128, 64, False), (128, 64, True)}
+
+
+def test_ragged_shapes_cover_every_launch_class(ops):
+    for fmt in (0, 1):
+        seen = set()
+        for M, N, K in RAGGED:
+            tm, tn, sp = ops.gemm_plan(M, N, K, fmt)
+            seen.add((tm, tn, sp > 1))
+        assert seen == LAUNCH_CLASSES, LAUNCH_CLASSES - seen
 
 
 @pytest.mark.parametrize("M,N,K", RAGGED)
