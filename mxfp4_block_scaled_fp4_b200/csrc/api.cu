@@ -129,20 +129,12 @@ fp4_status_t fp4_quantize_act(const void* x, int rows, int K, fp4_format_t fmt,
   a.g = g;
   a.codes = codes;
   a.scales = scales;
-  if (dyn) {
-    int used = 0;
-    unsigned* partial = static_cast<unsigned*>(ws);
-    if (fp4::launch_amax(x, static_cast<long long>(rows) * K, partial, &used, s, true) !=
-        cudaSuccess)
-      return FP4_ERR_CUDA;
-    a.partial = partial;
-    a.n_partial = used;
-  }
-  // Both passes are programmatic dependents of the kernel before them (each
-  // waits for its predecessor before reading), so their launches overlap
-  // the predecessor's tail.  The quantize pass does not release its own
-  // dependent early: a fused GEMM may read weights before its wait.
-  return from_cuda(fp4::launch_quantize(a, s, true));
+  // The amax pass (DYNAMIC) and the quantize pass, each a programmatic
+  // dependent of the kernel before it (each waits for its predecessor before
+  // reading), so its launch overlaps the predecessor's tail.  No pass
+  // releases its own dependent early: a fused GEMM may read weights before
+  // its wait.
+  return from_cuda(fp4::launch_quantize_act(a, static_cast<unsigned*>(ws), s));
 }
 
 fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt, uint8_t* codes,

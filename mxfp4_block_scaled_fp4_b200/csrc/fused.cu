@@ -453,16 +453,7 @@ cudaError_t launch_gemm_fused(const FusedArgs& f, cudaStream_t s) {
   q.zero_pad_rows = 0;
   // the GEMM reads the quantized activation only after its wait
   q.release_early = 1;
-  cudaError_t e;
-  if (f.dynamic) {
-    int used = 0;
-    e = launch_amax(f.a, static_cast<long long>(f.M) * f.K,
-                    reinterpret_cast<unsigned*>(ws + pl.off_partial), &used, s, true);
-    if (e != cudaSuccess) return e;
-    q.partial = reinterpret_cast<unsigned*>(ws + pl.off_partial);
-    q.n_partial = used;
-  }
-  e = launch_quantize(q, s, true);
+  cudaError_t e = launch_quantize_act(q, reinterpret_cast<unsigned*>(ws + pl.off_partial), s);
   if (e != cudaSuccess) return e;
 
   // 3: the swap-AB GEMM

@@ -53,6 +53,14 @@ struct QuantArgs {
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl = false);
 
+// Activation quantization: the amax pass (DYNAMIC; partial maxima into
+// `partial`, kAmaxSlots entries) and the quantize pass, each a programmatic
+// dependent of the kernel before it.  (One kernel on one thread-block
+// cluster, reducing the amax over distributed shared memory, measured
+// slower on B200 for every size: 16 SMs cannot match the full chip's
+// bandwidth, and two launches cost ~5 us whatever the size.)
+cudaError_t launch_quantize_act(QuantArgs a, unsigned* partial, cudaStream_t s);
+
 struct GemmArgs {
   const uint8_t* a_codes; const uint8_t* a_scales; const float* g_a;
   const uint8_t* w_codes; const uint8_t* w_scales; const float* g_w;

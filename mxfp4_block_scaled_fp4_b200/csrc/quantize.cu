@@ -113,10 +113,91 @@ __device__ __forceinline__ unsigned fast_div(unsigned n, FastDiv f) {
   return static_cast<unsigned>((static_cast<unsigned long long>(__umulhi(n, f.m)) + n) >> f.l);
 }
 
-// A warp quantizes a slab of 4 x 32 consecutive units per iteration: every
-// lane issues its 8 loads (4 units x 32 bytes) before computing.  With a
-// DYNAMIC global scale the slabs are walked from the end, so the first ones
-// are still in L2 from the amax pass.
+// Units [u_begin, u_end) in slabs of 4 x 32 consecutive units: warp w of
+// nwarps takes slabs w, w + nwarps, ... (from the end when `reverse`), and
+// every lane issues its 8 loads (4 units x 32 bytes) before computing.
+template <int FMT, int LAYOUT>
+__device__ __forceinline__ void quantize_units(const QuantArgs& a, long long u_begin,
+                                               long long u_end, long long w, long long nwarps,
+                                               bool reverse, int upr, FastDiv upr_div, int nsf,
+                                               int ncb, float six_g, float y6, bool fast_b,
+                                               const float* r_tab) {
+  const bool big = u_end > 0xFFFFFFFFll;   // unit indices beyond 32 bits: plain division
+  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
+  uint2* __restrict__ codes = reinterpret_cast<uint2*>(a.codes);
+  uint8_t* __restrict__ scales = a.scales;
+  const int lane = threadIdx.x & 31;
+  const long long n_slabs = (u_end - u_begin + 127) / 128;
+  for (long long t = w; t < n_slabs; t += nwarps) {
+    const long long slab = reverse ? n_slabs - 1 - t : t;
+    uint4 xs[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long long u = u_begin + slab * 128 + j * 32 + lane;
+      if (u < u_end) {
+        xs[j][0] = ld_stream(x + u * 16);
+        xs[j][1] = ld_stream(x + u * 16 + 8);
+      } else {
+        xs[j][0] = xs[j][1] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long long u = u_begin + slab * 128 + j * 32 + lane;
+      const uint4 p = xs[j][0], q = xs[j][1];
+      unsigned m = fold_u16x2(max_u16x2(mag_max8(p), mag_max8(q)));
+      unsigned sbyte;
+      uint2 packed;
+      float r;
+      if (FMT == 0) {
+        sbyte = nvfp4_scale_byte(m, six_g, y6, fast_b);
+        r = r_tab[sbyte & 127u];
+        packed = (r == 0.0f) ? make_uint2(0, 0)
+                             : make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
+      } else {
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));   // 32-value block = lane pair
+        sbyte = mxfp4_scale(m, &r);
+        packed = make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
+      }
+      if (u < u_end) {
+        codes[u] = packed;
+        const long long row =
+            big ? u / upr : static_cast<long long>(fast_div(static_cast<unsigned>(u), upr_div));
+        const int jj = static_cast<int>(u - row * upr);
+        if (FMT == 0 || (jj & 1) == 0) {
+          const int c = (FMT == 0) ? jj : (jj >> 1);
+          const long long off = (LAYOUT == 1) ? row * nsf + c : mma_scale_offset(row, c, ncb);
+          scales[off] = static_cast<uint8_t>(sbyte);
+        }
+      }
+    }
+  }
+}
+
+// MMA order: zero the padding, columns [nsf, 4 ncb) of real rows, then every
+// column of rows [rows, rows padded to 128); items i = first, first + stride...
+__device__ __forceinline__ void zero_mma_padding(const QuantArgs& a, long long pad_a,
+                                                 long long pad_b, int nsf, int ncb,
+                                                 long long first, long long stride) {
+  const long long total = pad_a + pad_b;
+  const int padc = 4 * ncb - nsf;
+  for (long long i = first; i < total; i += stride) {
+    long long r;
+    int c;
+    if (i < pad_a) {
+      r = i / padc;
+      c = nsf + static_cast<int>(i - r * padc);
+    } else {
+      const long long k = i - pad_a;
+      r = a.rows + k / (4 * ncb);
+      c = static_cast<int>(k % (4 * ncb));
+    }
+    a.scales[mma_scale_offset(r, c, ncb)] = 0;
+  }
+}
+
+// The full-chip quantize pass.  With a DYNAMIC global scale the slabs are
+// walked from the end, so the first ones are still in L2 from the amax pass.
 template <int FMT, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long long units,
                                                                int upr, FastDiv upr_div, int nsf,
@@ -135,81 +216,13 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long
     for (int i = threadIdx.x; i < 128; i += blockDim.x) r_tab[i] = nvfp4_recip(i, g);
     __syncthreads();
   }
-  const bool big = units > 0xFFFFFFFFll;   // unit indices beyond 32 bits: plain division
-
-  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
-  uint2* __restrict__ codes = reinterpret_cast<uint2*>(a.codes);
-  uint8_t* __restrict__ scales = a.scales;
-  const int lane = threadIdx.x & 31;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  const long long n_slabs = (units + 127) / 128;
   const long long gwarp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const long long nwarps = stride >> 5;
-  const bool reverse = a.dynamic != 0;
-  for (long long t = gwarp; t < n_slabs; t += nwarps) {
-    const long long slab = reverse ? n_slabs - 1 - t : t;
-    uint4 xs[4][2];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const long long u = slab * 128 + j * 32 + lane;
-      if (u < units) {
-        xs[j][0] = ld_stream(x + u * 16);
-        xs[j][1] = ld_stream(x + u * 16 + 8);
-      } else {
-        xs[j][0] = xs[j][1] = make_uint4(0, 0, 0, 0);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const long long u = slab * 128 + j * 32 + lane;
-      const uint4 p = xs[j][0], q = xs[j][1];
-      unsigned m = fold_u16x2(max_u16x2(mag_max8(p), mag_max8(q)));
-      unsigned sbyte;
-      uint2 packed;
-      float r;
-      if (FMT == 0) {
-        sbyte = nvfp4_scale_byte(m, six_g, y6, fast_b);
-        r = r_tab[sbyte & 127u];
-        packed = (r == 0.0f) ? make_uint2(0, 0)
-                             : make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
-      } else {
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));   // 32-value block = lane pair
-        sbyte = mxfp4_scale(m, &r);
-        packed = make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
-      }
-      if (u < units) {
-        codes[u] = packed;
-        const long long row =
-            big ? u / upr : static_cast<long long>(fast_div(static_cast<unsigned>(u), upr_div));
-        const int jj = static_cast<int>(u - row * upr);
-        if (FMT == 0 || (jj & 1) == 0) {
-          const int c = (FMT == 0) ? jj : (jj >> 1);
-          const long long off = (LAYOUT == 1) ? row * nsf + c : mma_scale_offset(row, c, ncb);
-          scales[off] = static_cast<uint8_t>(sbyte);
-        }
-      }
-    }
-  }
-  if (LAYOUT == 0) {
-    // zero the padding of the MMA order: columns [nsf, 4 ncb) of real rows,
-    // then every column of rows [rows, rows padded to 128)
-    const long long total = pad_a + pad_b;
-    const int padc = 4 * ncb - nsf;
-    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-         i += stride) {
-      long long r;
-      int c;
-      if (i < pad_a) {
-        r = i / padc;
-        c = nsf + static_cast<int>(i - r * padc);
-      } else {
-        const long long k = i - pad_a;
-        r = a.rows + k / (4 * ncb);
-        c = static_cast<int>(k % (4 * ncb));
-      }
-      scales[mma_scale_offset(r, c, ncb)] = 0;
-    }
-  }
+  quantize_units<FMT, LAYOUT>(a, 0, units, gwarp, stride >> 5, a.dynamic != 0, upr, upr_div, nsf,
+                              ncb, six_g, y6, fast_b, r_tab);
+  if (LAYOUT == 0)
+    zero_mma_padding(a, pad_a, pad_b, nsf, ncb,
+                     static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x, stride);
 }
 
 }  // namespace
@@ -256,33 +269,61 @@ cudaError_t launch_amax(const void* x, long long n, unsigned* partial, int* n_us
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl) {
-  const int upr = a.K / 16;
-  const long long units = a.rows * upr;
-  const int nsf = nsf_of(a.K, a.fmt);
-  const int ncb = ncb_of(nsf);
-  long long pad_a = 0, pad_b = 0;
+namespace {
+
+struct QuantGeom {
+  int upr, nsf, ncb;
+  long long units, pad_a, pad_b;
+  FastDiv fd;
+};
+
+QuantGeom quant_geom(const QuantArgs& a) {
+  QuantGeom q;
+  q.upr = a.K / 16;
+  q.units = a.rows * q.upr;
+  q.nsf = nsf_of(a.K, a.fmt);
+  q.ncb = ncb_of(q.nsf);
+  q.pad_a = q.pad_b = 0;
   if (a.layout == 0) {
-    pad_a = a.rows * (4 * ncb - nsf);
-    pad_b = a.zero_pad_rows ? (rows_pad128(a.rows) - a.rows) * 4 * ncb : 0;
+    q.pad_a = a.rows * (4 * q.ncb - q.nsf);
+    q.pad_b = a.zero_pad_rows ? (rows_pad128(a.rows) - a.rows) * 4 * q.ncb : 0;
   }
-  const long long want = std::max((units + kThreads * 4 - 1) / (kThreads * 4),
-                                  (pad_a + pad_b + kThreads - 1) / kThreads);
+  q.fd = FastDiv{0u, 0u};
+  if (q.upr > 1) {
+    unsigned l = 0;
+    while ((1ull << l) < static_cast<unsigned long long>(q.upr)) ++l;
+    q.fd.l = l;
+    q.fd.m = static_cast<unsigned>(((1ull << 32) * ((1ull << l) - static_cast<unsigned long long>(q.upr))) /
+                                       static_cast<unsigned long long>(q.upr) + 1);
+  }
+  return q;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl) {
+  const QuantGeom q = quant_geom(a);
+  const long long want = std::max((q.units + kThreads * 4 - 1) / (kThreads * 4),
+                                  (q.pad_a + q.pad_b + kThreads - 1) / kThreads);
   const int blocks = static_cast<int>(
       std::max<long long>(1, std::min<long long>(want, static_cast<long long>(sm_count()) * 4)));
   auto kern = (a.fmt == 0) ? (a.layout == 0 ? quantize_kernel<0, 0> : quantize_kernel<0, 1>)
                            : (a.layout == 0 ? quantize_kernel<1, 0> : quantize_kernel<1, 1>);
-  FastDiv fd{0u, 0u};
-  if (upr > 1) {
-    unsigned l = 0;
-    while ((1ull << l) < static_cast<unsigned long long>(upr)) ++l;
-    fd.l = l;
-    fd.m = static_cast<unsigned>(((1ull << 32) * ((1ull << l) - static_cast<unsigned long long>(upr))) /
-                                     static_cast<unsigned long long>(upr) + 1);
-  }
-  const cudaError_t e = launch_k(kern, blocks, pdl, s, a, units, upr, fd, nsf, ncb, pad_a, pad_b);
+  const cudaError_t e =
+      launch_k(kern, blocks, pdl, s, a, q.units, q.upr, q.fd, q.nsf, q.ncb, q.pad_a, q.pad_b);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_act(QuantArgs a, unsigned* partial, cudaStream_t s) {
+  if (a.dynamic) {
+    int used = 0;
+    const cudaError_t e = launch_amax(a.x, a.rows * a.K, partial, &used, s, true);
+    if (e != cudaSuccess) return e;
+    a.partial = partial;
+    a.n_partial = used;
+  }
+  return launch_quantize(a, s, true);
 }
 
 }  // namespace fp4
