@@ -45,6 +45,16 @@ FP4_OVER_BF16 = 4.0     # nominal dense FP4 / dense BF16 tensor throughput on B2
 GEMM_TRAFFIC_BYTES = 306.7e6 + 435.2e6
 
 
+def gemm_kernel_name(m, n, k):
+    """The GEMM kernel fp4_gemm launches for this shape (fp4_gemm_plan)."""
+    from mxfp4_block_scaled_fp4_b200 import ops
+    tm, tn, sp = ops.gemm_plan(m, n, k, 0)
+    if tm == 256:
+        return "fp4 gemm_pair_kernel (tcgen05 cta_group::2 kind::mxf4nvf4, 256x256 tiles)"
+    return (f"fp4 gemm_kernel (tcgen05 cta_group::1 kind::mxf4nvf4, {tm}x{tn} tiles"
+            + (f", K split over {sp}-CTA clusters)" if sp > 1 else ")"))
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -533,7 +543,7 @@ def main():
                      "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
                      "traffic": GEMM_TRAFFIC_BYTES if (M, N, K) == (8192, 28672, 8192) else None,
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read + write)",
-                     "kernel": "fp4 gemm_pair_kernel (tcgen05 cta_group::2 kind::mxf4nvf4)",
+                     "kernel": gemm_kernel_name(M, N, K),
                      "peak_source": f"{src} bf16_tflops_sustained x {FP4_OVER_BF16:g} "
                                     "(nominal dense FP4/BF16 ratio)"},
         "quantize": {"achieved_gbs": q_gbs, "peak_gbs": peaks["hbm_gbs"],
