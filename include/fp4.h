@@ -123,6 +123,9 @@ fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt,
  * accumulated in FP32 in tensor memory; C = RN(alpha * acc) is written as
  * bf16 (round to nearest even) or fp32, row-major with leading dimension
  * ldc (elements).  Any M >= 0 (no padding asked of the caller), N % 8 == 0.
+ * The launch shape follows the problem (fp4_gemm_plan): when output tiles
+ * are few, K may be split over a thread-block cluster whose partial sums are
+ * added in a fixed order, so repeated calls give identical bits.
  * The pages' W4A4 GEMM: "fp4-cuda-kernel" forum post; cuBLAS's refusal of
  * M < 128 that this entry point does not share: "Hardware FP4 inference for
  * speech on Blackwell", section "Do the FP4 tensor cores even engage?". */

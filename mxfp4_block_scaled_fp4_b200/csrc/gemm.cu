@@ -548,8 +548,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       // own rows written by all four warps; peers' rows by their st.async
       asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (acc_ok && hi > lo &&
-          __all_sync(0xFFFFFFFFu, mbar_wait(recv, 0, abort_flag, p.watchdog, WD_EPILOGUE))) {
+      const bool got = acc_ok && hi > lo &&
+                       __all_sync(0xFFFFFFFFu, mbar_wait(recv, 0, abort_flag, p.watchdog, WD_EPILOGUE));
+      if (!got && hi > lo && tid == 0) {
+        // unwinding: the peers' pushes may still be in flight into this
+        // CTA's shared memory; let them land (bounded) before it goes away
+        mbar_wait_drain(recv, 0, p.watchdog);
+      }
+      if (got) {
         // 2) the owned rows: (row, 8-column group) units shared out, rows
         // fastest so that a warp's shared-memory reads are contiguous
         const int rows = hi - lo;

@@ -82,6 +82,21 @@ def test_ragged_shapes(ops, orc, M, N, K, fmt, dt):
     run_pair(ops, orc, a, w, fmt, dt)
 
 
+@pytest.mark.parametrize("M,N,K", [(8, 720, 7680), (256, 2880, 7680), (200, 1024, 6400)])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_split_k_is_deterministic(ops, M, N, K, fmt):
+    """K split over a cluster: the partial sums are added in split order, so
+    repeated calls give identical bits."""
+    assert ops.gemm_plan(M, N, K, fmt)[2] > 1
+    a = inputs.random_bf16(300 + M, (M, K)).cuda()
+    w = inputs.random_bf16(400 + N, (N, K), 0.02).cuda()
+    aq = ops.quantize(a, fmt, ops.SCALES_MMA)
+    wq = ops.quantize_weights(w, fmt)
+    outs = [ops.gemm(aq, wq, torch.float32) for _ in range(4)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+
+
 @pytest.mark.parametrize("M", [1, 8, 32])
 @pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096), (4096, 14336)])
 def test_decode_shapes_fused(ops, orc, M, N, K):
