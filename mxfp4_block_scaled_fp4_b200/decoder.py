@@ -25,6 +25,12 @@ whether FP4 buys speed at small batch).
 
 The bf16 reference runs the same layer structure with torch matmuls
 (cuBLAS), gate/up/down each as one GEMM over the concatenated weights.
+
+Both forwards run the projections that share an input as concurrent
+branches of the graph (side streams forked from and joined back into the
+caller's stream): q | k | v, then gate0 | gate1 | up0 | up1 (bf16: gate |
+up), then down0 .. down3 (bf16: one GEMM).  At decode sizes each call is
+mostly fixed latency, which the branches overlap.
 """
 from __future__ import annotations
 
@@ -70,14 +76,48 @@ class SyntheticDecoder:
             self.wq.append(qd)
             self.wb.append(bd)
         self.record = None   # list of (layer, name, input, output) when set to a list
+        # side streams for the concurrent branches of a layer, and one
+        # library workspace per branch (concurrent calls must not share one)
+        self.side = [torch.cuda.Stream(device=self.device) for _ in range(3)]
+        self.ws = [None] * 4
+        self.branch = 0   # index of the branch the next _gemm call runs in
+
+    def _branches(self, fns):
+        """Run fns[0] on the current stream and fns[i] on side stream i-1,
+        all after the work already queued, and join them back."""
+        cur = torch.cuda.current_stream(self.device)
+        for s in self.side[:len(fns) - 1]:
+            s.wait_stream(cur)
+        outs = [None] * len(fns)
+        for i, fn in enumerate(fns[1:]):
+            with torch.cuda.stream(self.side[i]):
+                self.branch = i + 1
+                outs[i + 1] = fn()
+        self.branch = 0
+        outs[0] = fns[0]()
+        for s in self.side[:len(fns) - 1]:
+            cur.wait_stream(s)
+        return outs
+
+    def _ws(self, M: int, N: int, K: int) -> torch.Tensor:
+        """This branch's workspace, grown outside graph capture only (the
+        forward runs eagerly before it is captured)."""
+        need = ops.L.fp4_workspace_bytes(M, N, K, self.fmt)
+        b = self.branch
+        if self.ws[b] is None or self.ws[b].numel() < need:
+            if torch.cuda.is_current_stream_capturing():
+                raise RuntimeError("decoder workspace must be sized before capture")
+            self.ws[b] = torch.empty(max(need, 1 << 16), dtype=torch.uint8, device=self.device)
+        return self.ws[b]
 
     # ------------------------------------------------------------ FP4 path
     def _gemm(self, li: int, name: str, x: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
         w = self.wq[li][name]
+        ws = self._ws(x.shape[0], w.rows, w.K)
         if x.shape[0] <= 32:
-            ops.gemm_fused(x, w, out=out)
+            ops.gemm_fused(x, w, out=out, ws=ws)
         else:
-            ops.gemm(ops.quantize(x, self.fmt, ops.SCALES_MMA), w, out=out)
+            ops.gemm(ops.quantize(x, self.fmt, ops.SCALES_MMA, ws=ws), w, out=out)
         if self.record is not None:
             self.record.append((li, name, x.clone(), out.clone()))
         return out
@@ -87,22 +127,25 @@ class SyntheticDecoder:
         dev = x.device
         bf = torch.bfloat16
         for li in range(self.layers):
-            t = torch.empty((M, HIDDEN), dtype=bf, device=dev)
-            self._gemm(li, "q", x, t)
-            self._gemm(li, "k", x, t)
-            v = self._gemm(li, "v", x, torch.empty((M, HIDDEN), dtype=bf, device=dev))
+            tq = torch.empty((M, HIDDEN), dtype=bf, device=dev)
+            tk = torch.empty((M, HIDDEN), dtype=bf, device=dev)
+            v = torch.empty((M, HIDDEN), dtype=bf, device=dev)
+            self._branches([lambda: self._gemm(li, "v", x, v),
+                            lambda: self._gemm(li, "q", x, tq),
+                            lambda: self._gemm(li, "k", x, tk)])
             o = self._gemm(li, "o", v, torch.empty((M, HIDDEN), dtype=bf, device=dev))
             x = (x + o) * RES
             gate = torch.empty((M, FFN), dtype=bf, device=dev)
             up = torch.empty((M, FFN), dtype=bf, device=dev)
-            for i in range(2):
-                self._gemm(li, f"gate{i}", x, gate[:, i * (FFN // 2):(i + 1) * (FFN // 2)])
-            for i in range(2):
-                self._gemm(li, f"up{i}", x, up[:, i * (FFN // 2):(i + 1) * (FFN // 2)])
+            half = FFN // 2
+            self._branches([lambda i=i, t=t, name=name: self._gemm(li, f"{name}{i}", x,
+                                                                   t[:, i * half:(i + 1) * half])
+                            for name, t in (("gate", gate), ("up", up)) for i in range(2)])
             h = torch.nn.functional.silu(gate) * up
             down = torch.empty((M, HIDDEN), dtype=bf, device=dev)
-            for i in range(4):
-                self._gemm(li, f"down{i}", h, down[:, i * (HIDDEN // 4):(i + 1) * (HIDDEN // 4)])
+            q4 = HIDDEN // 4
+            self._branches([lambda i=i: self._gemm(li, f"down{i}", h, down[:, i * q4:(i + 1) * q4])
+                            for i in range(4)])
             x = (x + down) * RES
         return x
 
@@ -110,11 +153,11 @@ class SyntheticDecoder:
     def forward_bf16(self, x: torch.Tensor) -> torch.Tensor:
         for li in range(self.layers):
             W = self.wb[li]
-            x @ W["q"].T
-            x @ W["k"].T
-            v = x @ W["v"].T
+            v, _, _ = self._branches([lambda: x @ W["v"].T, lambda: x @ W["q"].T,
+                                      lambda: x @ W["k"].T])
             x = (x + v @ W["o"].T) * RES
-            h = torch.nn.functional.silu(x @ W["gate"].T) * (x @ W["up"].T)
+            g, u = self._branches([lambda: x @ W["gate"].T, lambda: x @ W["up"].T])
+            h = torch.nn.functional.silu(g) * u
             x = (x + h @ W["down"].T) * RES
         return x
 

@@ -59,8 +59,11 @@ class Quantized:
 
 
 def quantize(x: torch.Tensor, fmt: int = NVFP4, layout: int = SCALES_MMA,
-             g: torch.Tensor | None = None) -> Quantized:
-    """fp4_quantize_act: DYNAMIC global scale when g is None, else STATIC g."""
+             g: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> Quantized:
+    """fp4_quantize_act: DYNAMIC global scale when g is None, else STATIC g.
+    ws: scratch of at least fp4_workspace_bytes bytes; calls that may run
+    concurrently (other streams) need their own, else the shared per-device
+    buffer is used."""
     _cuda_bf16_2d(x, "x")
     rows, K = x.shape
     dev = x.device
@@ -70,7 +73,10 @@ def quantize(x: torch.Tensor, fmt: int = NVFP4, layout: int = SCALES_MMA,
     gmode = L.FP4_GLOBAL_DYNAMIC if g is None else L.FP4_GLOBAL_STATIC
     gt = torch.ones(1, dtype=torch.float32, device=dev) if g is None else g
     ws_bytes = L.fp4_workspace_bytes(rows, 0, K, fmt)
-    ws = workspace(ws_bytes, dev)
+    if ws is None:
+        ws = workspace(ws_bytes, dev)
+    elif ws.numel() < ws_bytes:
+        raise ValueError("workspace too small")
     _check(L.fp4_quantize_act(x.data_ptr(), rows, K, fmt, layout, gmode, gt.data_ptr(),
                               codes.data_ptr(), scales.data_ptr(), ws.data_ptr(), ws.numel(),
                               _stream()), "fp4_quantize_act")
@@ -119,8 +125,9 @@ def gemm_plan(M: int, N: int, K: int, fmt: int = NVFP4) -> tuple[int, int, int]:
 
 def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
                g_a: torch.Tensor | None = None, out: torch.Tensor | None = None,
-               g_out: torch.Tensor | None = None) -> torch.Tensor:
-    """fp4_gemm_fused: quantize x (M <= 32) on the fly and multiply with w."""
+               g_out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """fp4_gemm_fused: quantize x (M <= 32) on the fly and multiply with w.
+    ws: as for quantize (concurrent calls need their own)."""
     _cuda_bf16_2d(x, "x")
     M, K = x.shape
     N = w.rows
@@ -131,7 +138,11 @@ def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
     gmode = L.FP4_GLOBAL_DYNAMIC if g_a is None else L.FP4_GLOBAL_STATIC
     if g_a is None:
         g_a = g_out if g_out is not None else torch.ones(1, dtype=torch.float32, device=dev)
-    ws = workspace(L.fp4_workspace_bytes(M, N, K, w.fmt), dev)
+    need = L.fp4_workspace_bytes(M, N, K, w.fmt)
+    if ws is None:
+        ws = workspace(need, dev)
+    elif ws.numel() < need:
+        raise ValueError("workspace too small")
     _check(L.fp4_gemm_fused(x.data_ptr(), w.codes.data_ptr(), w.scales.data_ptr(),
                             w.g.data_ptr(), M, N, K, w.fmt, gmode, g_a.data_ptr(),
                             out.data_ptr(), out.stride(0), o, ws.data_ptr(), ws.numel(),
