@@ -335,6 +335,8 @@ def measure_decoder(torch, dev, batch_sizes=(1, 16, 256), reps=20):
             del g
         row["speedup_vs_bf16"] = round(row["us_per_forward_bf16"] / row["us_per_forward_fp4"], 3)
         row["fp4_weight_bytes"] = dec.weight_bytes()
+        row["structure"] = ("per layer q|k|v, o, gate0|gate1|up0|up1, down0..3 as concurrent "
+                            "graph branches; bf16: q|k|v, o, gate|up, down")
         res.append(row)
     return res
 
