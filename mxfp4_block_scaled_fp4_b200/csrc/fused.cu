@@ -245,8 +245,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       for (int i = 0; i < n_steps && ok; ++i) {
         const int stage = i % FSTAGES;
         const uint32_t phase = static_cast<uint32_t>(i / FSTAGES) & 1u;
-        ok = mbar_wait(&full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL) &&
-             mbar_wait(&sf_full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL);
+        // one wait per step: the staging warps arrive on sf_full only after
+        // the step's weight tile has landed (a test of an mbarrier is a
+        // ~250-cycle round trip even when its phase has completed)
+        ok = mbar_wait(&sf_full[stage], phase, abort_flag, p.watchdog, WD_MMA_FULL);
         if (!ok) break;
         tc_fence_after();
         const int kglob = (s_lo + i) * FBK;
