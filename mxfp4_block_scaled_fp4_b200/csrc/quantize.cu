@@ -43,12 +43,28 @@ __device__ __forceinline__ long long mma_scale_offset(long long r, int c, int nc
 
 // Global scale from the partial maxima of the amax pass (DYNAMIC), or the
 // caller's value (STATIC).  g = amax / 2688, 1 for an all-zero tensor.
+// self_amax: the maximum over the whole tensor x (n_vec 16-byte vectors)
+// instead of the partial maxima (small tensors; 4 loads in flight a thread).
 __device__ float global_scale(int dynamic, const float* g, const unsigned* partial,
-                              int n_partial) {
+                              int n_partial, int self_amax, const uint4* x, long long n_vec) {
   if (!dynamic) return *g;
   __shared__ unsigned red[kThreads / 32];
   unsigned m = 0;
-  for (int i = threadIdx.x; i < n_partial; i += blockDim.x) m = max(m, partial[i]);
+  if (self_amax) {
+    for (long long i = threadIdx.x; i < n_vec; i += 4 * blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const long long k = i + j * blockDim.x;
+        v[j] = (k < n_vec) ? ld_stream(x + k) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m = max_u16x2(m, mag_max8(v[j]));
+    }
+    m = fold_u16x2(m);
+  } else {
+    for (int i = threadIdx.x; i < n_partial; i += blockDim.x) m = max(m, partial[i]);
+  }
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
@@ -205,7 +221,9 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long
                                                                long long pad_b) {
   if (a.release_early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const float g = (FMT == 0) ? global_scale(a.dynamic, a.g, a.partial, a.n_partial) : 1.0f;
+  const float g = (FMT == 0) ? global_scale(a.dynamic, a.g, a.partial, a.n_partial, a.self_amax,
+                                            static_cast<const uint4*>(a.x), units * 2)
+                             : 1.0f;
   if (FMT == 0 && a.dynamic && blockIdx.x == 0 && threadIdx.x == 0) *a.g = g;
   const float six_g = __fmul_rn(6.0f, g);
   const float y6 = __frcp_rn(six_g);
@@ -316,6 +334,10 @@ cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl) {
 }
 
 cudaError_t launch_quantize_act(QuantArgs a, unsigned* partial, cudaStream_t s) {
+  if (a.dynamic && a.rows * a.K * 2 <= kSelfAmaxBytes) {
+    a.self_amax = 1;
+    return launch_quantize(a, s, true);
+  }
   if (a.dynamic) {
     int used = 0;
     const cudaError_t e = launch_amax(a.x, a.rows * a.K, partial, &used, s, true);

@@ -57,6 +57,13 @@ def test_mxfp4_sweep(ops, orc, M, K):
     check_quant(ops, orc, act(M, K), 1)
 
 
+# DYNAMIC tensors of at most 32 KiB skip the amax pass (each quantize CTA
+# reads the whole tensor for its global scale); either side of that limit
+@pytest.mark.parametrize("M,K", [(1, 16384), (1, 16416), (2, 8192), (2, 8224)])
+def test_nvfp4_dynamic_self_amax_limit(ops, orc, M, K):
+    check_quant(ops, orc, inputs.act_sweep(M, K), 0)
+
+
 @pytest.mark.parametrize("M,K", [(32, 2880), (512, 8192)])
 @pytest.mark.parametrize("g", [1.0, 0.0123])
 def test_nvfp4_static_global_scale(ops, orc, M, K, g):
