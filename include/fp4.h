@@ -136,10 +136,17 @@ fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const flo
                       void* ws, size_t ws_bytes, void* stream);
 
 /* Small-M path (decode): quantize the bf16 activation a [M, K] on the fly
- * and multiply it with pre-quantized weights, as one chain of programmatic
- * dependent launches on `stream`: amax (DYNAMIC only) -> quantize (into the
- * workspace) -> a swap-AB, split-K tcgen05 GEMM for M <= 32 that starts
- * streaming the weights before the quantized activation is ready.
+ * and multiply it with pre-quantized weights.  Small activations (M*K up to
+ * 32768 values) take ONE kernel: every CTA streams its weight tile from its
+ * first instruction, then takes the activation's global amax, quantizes its
+ * own K slice into shared memory and runs its MMAs.  Larger ones are a
+ * chain of programmatic dependent launches on `stream`: amax (DYNAMIC only)
+ * -> quantize (into the workspace) -> a swap-AB, split-K tcgen05 GEMM for
+ * M <= 32 that starts streaming the weights before the quantized activation
+ * is ready.  Either way the kernels may begin reading w_codes / w_scales
+ * before the kernel preceding them on `stream` has finished, so the
+ * weights must not be written by that kernel (quantize them earlier, as at
+ * load time, or synchronize the stream first).
  * "FP4 n'existe pas", runtime survey (quantization, scaling, matmul and
  * de-scaling chained in one go); the small-M regime: "Hardware FP4
  * inference for speech on Blackwell", section "Do the FP4 tensor cores even
