@@ -471,7 +471,7 @@ def main():
             ev_q1[i].record(stream)
         check(L.fp4_gemm(codes.data_ptr(), scales.data_ptr(), g_a.data_ptr(), wq.codes.data_ptr(),
                          wq.scales.data_ptr(), wq.g.data_ptr(), M, N, K, 0, c.data_ptr(), N, 0,
-                         ws.data_ptr(), ws_bytes, sp), "gemm")
+                         ws.data_ptr(), ws_bytes, 0, sp), "gemm")
         if timed:
             ev_g1[i].record(stream)
 

@@ -126,6 +126,10 @@ fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt,
  * The launch shape follows the problem (fp4_gemm_plan): when output tiles
  * are few, K may be split over a thread-block cluster whose partial sums are
  * added in a fixed order, so repeated calls give identical bits.
+ * max_sms: the SMs the launch shape is chosen for (0 = the whole device).
+ * A caller that runs several GEMMs at once on different streams gives each
+ * its share, so that their CTAs run side by side; it changes the tile width
+ * and K split (hence the FP32 summation order), never the arithmetic.
  * The pages' W4A4 GEMM: "fp4-cuda-kernel" forum post; cuBLAS's refusal of
  * M < 128 that this entry point does not share: "Hardware FP4 inference for
  * speech on Blackwell", section "Do the FP4 tensor cores even engage?". */
@@ -133,7 +137,7 @@ fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const flo
                       const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
                       int M, int N, int K, fp4_format_t fmt,
                       void* C, int ldc, fp4_out_t out,
-                      void* ws, size_t ws_bytes, void* stream);
+                      void* ws, size_t ws_bytes, int max_sms, void* stream);
 
 /* Small-M path (decode): quantize the bf16 activation a [M, K] on the fly
  * and multiply it with pre-quantized weights.  Small activations (M*K up to
@@ -190,9 +194,10 @@ fp4_status_t fp4_gemm_fused(const void* a, const uint8_t* w_codes, const uint8_t
  * along K: a thread-block cluster whose CTAs each accumulate one slice of K
  * and then add their FP32 partial sums in a fixed order (split 0 first), so
  * repeated calls give identical bits.  Narrow tiles and splits are taken
- * when 256-wide tiles would leave most SMs idle.  Errors as fp4_gemm's
- * shape checks, FP4_ERR_INVALID_ARG for a NULL output pointer. */
-fp4_status_t fp4_gemm_plan(int M, int N, int K, fp4_format_t fmt,
+ * when 256-wide tiles would leave most of the max_sms SMs (0 = all of the
+ * device's) idle.  Errors as fp4_gemm's shape checks, FP4_ERR_INVALID_ARG
+ * for a NULL output pointer or a negative max_sms. */
+fp4_status_t fp4_gemm_plan(int M, int N, int K, fp4_format_t fmt, int max_sms,
                            int* tile_m, int* tile_n, int* splits);
 
 fp4_status_t fp4_quantize_act_noalloc(const void* x, int rows, int K, fp4_format_t fmt,

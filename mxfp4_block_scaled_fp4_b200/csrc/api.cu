@@ -147,12 +147,13 @@ fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt,
 fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
                       const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, int M,
                       int N, int K, fp4_format_t fmt, void* C, int ldc, fp4_out_t out, void* ws,
-                      size_t ws_bytes, void* stream) {
+                      size_t ws_bytes, int max_sms, void* stream) {
   (void)ws;
   (void)ws_bytes;
   fp4_status_t st;
   if ((st = check_format(fmt)) != FP4_OK) return st;
   if (out != FP4_OUT_BF16 && out != FP4_OUT_F32) return FP4_ERR_INVALID_ARG;
+  if (max_sms < 0) return FP4_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (M == 0 || N == 0) return FP4_OK;   // nothing is read or written
@@ -180,18 +181,19 @@ fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const flo
   a.C = C;
   a.ldc = ldc;
   a.out_f32 = out == FP4_OUT_F32;
+  a.max_sms = max_sms;
   return from_cuda(fp4::launch_gemm(a, static_cast<cudaStream_t>(stream)));
 }
 
-fp4_status_t fp4_gemm_plan(int M, int N, int K, fp4_format_t fmt, int* tile_m, int* tile_n,
-                           int* splits) {
+fp4_status_t fp4_gemm_plan(int M, int N, int K, fp4_format_t fmt, int max_sms, int* tile_m,
+                           int* tile_n, int* splits) {
   fp4_status_t st;
   if ((st = check_format(fmt)) != FP4_OK) return st;
   if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
-  if (!tile_m || !tile_n || !splits) return FP4_ERR_INVALID_ARG;
+  if (!tile_m || !tile_n || !splits || max_sms < 0) return FP4_ERR_INVALID_ARG;
   if ((st = device_ok()) != FP4_OK) return st;
-  return from_cuda(fp4::gemm_plan(M, N, K, tile_m, tile_n, splits));
+  return from_cuda(fp4::gemm_plan(M, N, K, max_sms, tile_m, tile_n, splits));
 }
 
 fp4_status_t fp4_gemm_fused(const void* x, const uint8_t* w_codes, const uint8_t* w_scales,

@@ -765,6 +765,7 @@ bool takes_pair(int M, int N, int sms) {
 
 template <int BN>
 cudaError_t launch_bn(const GemmArgs& a, Params p, int splits, cudaStream_t s) {
+  const int sms = gemm_sms(a.max_sms);
   CUtensorMap ma, mw;
   if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, a.w_codes, a.N, a.K, BN)) return cudaErrorInvalidValue;
@@ -772,7 +773,7 @@ cudaError_t launch_bn(const GemmArgs& a, Params p, int splits, cudaStream_t s) {
   p.splits = splits;
   p.k_per = (p.k_steps + splits - 1) / splits;
   const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = (splits > 1) ? tiles * splits : std::max(1, std::min(tiles, sm_count()));
+  const int grid = (splits > 1) ? tiles * splits : std::max(1, std::min(tiles, sms));
   if (a.fmt == 0)
     return a.out_f32 ? launch_typed<0, 1, BN>(ma, mw, p, grid, s)
                      : launch_typed<0, 0, BN>(ma, mw, p, grid, s);
@@ -782,8 +783,13 @@ cudaError_t launch_bn(const GemmArgs& a, Params p, int splits, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
+int gemm_sms(int max_sms) {
   const int sms = sm_count();
+  return (max_sms > 0 && max_sms < sms) ? max_sms : sms;
+}
+
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  const int sms = gemm_sms(a.max_sms);
   if (takes_pair(a.M, a.N, sms)) return launch_gemm_pair(a, s);
   Params p;
   p.a_scales = a.a_scales;
@@ -807,8 +813,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   return launch_bn<256>(a, p, sh.splits, s);
 }
 
-cudaError_t gemm_plan(int M, int N, int K, int* tile_m, int* tile_n, int* splits) {
-  const int sms = sm_count();
+cudaError_t gemm_plan(int M, int N, int K, int max_sms, int* tile_m, int* tile_n, int* splits) {
+  const int sms = gemm_sms(max_sms);
   if (sms <= 0) return cudaErrorNoDevice;
   if (takes_pair(M, N, sms)) {
     *tile_m = 2 * BM;

@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int FMT, int OUT_F32>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc,
-                         const Params& p, int tiles, cudaStream_t s) {
+                         const Params& p, int tiles, int max_sms, cudaStream_t s) {
   auto kern = gemm_pair_kernel<FMT, OUT_F32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -536,7 +536,7 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUt
     if (n <= 0) return cudaErrorInvalidConfiguration;
     max_pairs[dev] = n;
   }
-  const int pairs = std::max(1, std::min(tiles, max_pairs[dev]));
+  const int pairs = std::max(1, std::min({tiles, max_pairs[dev], gemm_sms(max_sms) / 2}));
   cfg.gridDim = dim3(2 * pairs);
   e = cudaLaunchKernelEx(&cfg, kern, ma, mw, mc, p);
   if (e != cudaSuccess) return e;
@@ -573,10 +573,10 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
   if (!p.watchdog) return cudaErrorInvalidSymbol;
   const int tiles = p.m_tiles * p.n_tiles;
   if (a.fmt == 0)
-    return a.out_f32 ? launch_typed<0, 1>(ma, mw, mc, p, tiles, s)
-                     : launch_typed<0, 0>(ma, mw, mc, p, tiles, s);
-  return a.out_f32 ? launch_typed<1, 1>(ma, mw, mc, p, tiles, s)
-                   : launch_typed<1, 0>(ma, mw, mc, p, tiles, s);
+    return a.out_f32 ? launch_typed<0, 1>(ma, mw, mc, p, tiles, a.max_sms, s)
+                     : launch_typed<0, 0>(ma, mw, mc, p, tiles, a.max_sms, s);
+  return a.out_f32 ? launch_typed<1, 1>(ma, mw, mc, p, tiles, a.max_sms, s)
+                   : launch_typed<1, 0>(ma, mw, mc, p, tiles, a.max_sms, s);
 }
 
 }  // namespace fp4

@@ -76,10 +76,14 @@ struct GemmArgs {
   const uint8_t* w_codes; const uint8_t* w_scales; const float* g_w;
   int M, N, K, fmt;
   void* C; int ldc; int out_f32;
+  int max_sms;          // SMs the launch shape is chosen for, 0 = the device's
 };
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s);
 // The shape launch_gemm takes: tile rows x columns, CTAs per tile along K.
-cudaError_t gemm_plan(int M, int N, int K, int* tile_m, int* tile_n, int* splits);
+cudaError_t gemm_plan(int M, int N, int K, int max_sms, int* tile_m, int* tile_n, int* splits);
+// The SMs a GEMM's launch shape is chosen for: max_sms when 0 < max_sms <
+// the device's count, else the device's.
+int gemm_sms(int max_sms);
 // The CTA-pair kernel (256 x 256 tiles); launch_gemm takes it for M > 128
 // when its tiles keep at least half the SMs busy.
 cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s);

@@ -30,7 +30,9 @@ Both forwards run the projections that share an input as concurrent
 branches of the graph (side streams forked from and joined back into the
 caller's stream): q | k | v, then gate0 | gate1 | up0 | up1 (bf16: gate |
 up), then down0 .. down3 (bf16: one GEMM).  At decode sizes each call is
-mostly fixed latency, which the branches overlap.
+mostly fixed latency, which the branches overlap.  Each fp4_gemm of an
+n-way group chooses its launch shape for 1/n of the SMs (max_sms), so that
+the group's CTAs run side by side instead of queueing.
 """
 from __future__ import annotations
 
@@ -81,6 +83,10 @@ class SyntheticDecoder:
         self.side = [torch.cuda.Stream(device=self.device) for _ in range(3)]
         self.ws = [None] * 4
         self.branch = 0   # index of the branch the next _gemm call runs in
+        # the SMs each GEMM of an n-way branch group chooses its launch shape
+        # for (its share of the device; 0 = all, outside the groups)
+        self.sms = torch.cuda.get_device_properties(self.device).multi_processor_count
+        self.max_sms = 0
 
     def _branches(self, fns):
         """Run fns[0] on the current stream and fns[i] on side stream i-1,
@@ -89,6 +95,7 @@ class SyntheticDecoder:
         for s in self.side[:len(fns) - 1]:
             s.wait_stream(cur)
         outs = [None] * len(fns)
+        self.max_sms = self.sms // len(fns) if len(fns) > 1 else 0
         for i, fn in enumerate(fns[1:]):
             with torch.cuda.stream(self.side[i]):
                 self.branch = i + 1
@@ -97,6 +104,7 @@ class SyntheticDecoder:
         outs[0] = fns[0]()
         for s in self.side[:len(fns) - 1]:
             cur.wait_stream(s)
+        self.max_sms = 0
         return outs
 
     def _ws(self, M: int, N: int, K: int) -> torch.Tensor:
@@ -117,7 +125,8 @@ class SyntheticDecoder:
         if x.shape[0] <= 32:
             ops.gemm_fused(x, w, out=out, ws=ws)
         else:
-            ops.gemm(ops.quantize(x, self.fmt, ops.SCALES_MMA, ws=ws), w, out=out)
+            ops.gemm(ops.quantize(x, self.fmt, ops.SCALES_MMA, ws=ws), w, out=out,
+                     max_sms=self.max_sms)
         if self.record is not None:
             self.record.append((li, name, x.clone(), out.clone()))
         return out

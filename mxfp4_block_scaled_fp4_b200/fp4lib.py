@@ -58,9 +58,9 @@ SIGNATURES = {
     "fp4_workspace_bytes": (SZ, [I, I, I, I]),
     "fp4_quantize_act": (I, [P, I, I, I, I, I, FP, U8P, U8P, P, SZ, P]),
     "fp4_quantize_weights": (I, [P, I, I, I, U8P, U8P, FP, P, SZ, P]),
-    "fp4_gemm": (I, [U8P, U8P, FP, U8P, U8P, FP, I, I, I, I, P, I, I, P, SZ, P]),
+    "fp4_gemm": (I, [U8P, U8P, FP, U8P, U8P, FP, I, I, I, I, P, I, I, P, SZ, I, P]),
     "fp4_gemm_fused": (I, [P, U8P, U8P, FP, I, I, I, I, I, FP, P, I, I, P, SZ, P]),
-    "fp4_gemm_plan": (I, [I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
+    "fp4_gemm_plan": (I, [I, I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
     "fp4_quantize_act_noalloc": (I, [P, I, I, I, I, I, FP, U8P, U8P, P]),
     "fp4_device_status": (I, [ctypes.POINTER(ctypes.c_uint), P]),
     "fp4_watchdog_selftest": (I, [ctypes.c_ulonglong, P]),
@@ -119,9 +119,9 @@ def fp4_quantize_weights(w, N, K, fmt, codes, scales, g, ws, ws_bytes, stream):
 
 
 def fp4_gemm(a_codes, a_scales, g_a, w_codes, w_scales, g_w, M, N, K, fmt, C, ldc, out, ws,
-             ws_bytes, stream):
+             ws_bytes, max_sms, stream):
     return _call("fp4_gemm", a_codes, a_scales, g_a, w_codes, w_scales, g_w, M, N, K, fmt, C,
-                 ldc, out, ws, ws_bytes, stream)
+                 ldc, out, ws, ws_bytes, max_sms, stream)
 
 
 def fp4_gemm_fused(a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc, out, ws,
@@ -130,8 +130,8 @@ def fp4_gemm_fused(a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc, 
                  out, ws, ws_bytes, stream)
 
 
-def fp4_gemm_plan(M, N, K, fmt, tile_m, tile_n, splits):
-    return _call("fp4_gemm_plan", M, N, K, fmt, tile_m, tile_n, splits)
+def fp4_gemm_plan(M, N, K, fmt, max_sms, tile_m, tile_n, splits):
+    return _call("fp4_gemm_plan", M, N, K, fmt, max_sms, tile_m, tile_n, splits)
 
 
 def fp4_quantize_act_noalloc(x, rows, K, fmt, layout, gmode, g, codes, scales, stream):

@@ -100,8 +100,9 @@ def quantize_weights(w: torch.Tensor, fmt: int = NVFP4) -> Quantized:
 
 
 def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
-         out: torch.Tensor | None = None) -> torch.Tensor:
-    """fp4_gemm: C = alpha * A_hat . W_hat^T."""
+         out: torch.Tensor | None = None, max_sms: int = 0) -> torch.Tensor:
+    """fp4_gemm: C = alpha * A_hat . W_hat^T.  max_sms: the SMs the launch
+    shape is chosen for (0 = all; concurrent GEMMs each take a share)."""
     if a.fmt != w.fmt or a.K != w.K or a.layout != SCALES_MMA or w.layout != SCALES_MMA:
         raise ValueError("operands must share format and K and use the MMA scale layout")
     M, N, K = a.rows, w.rows, a.K
@@ -111,15 +112,15 @@ def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
     o = L.FP4_OUT_F32 if out.dtype == torch.float32 else L.FP4_OUT_BF16
     _check(L.fp4_gemm(a.codes.data_ptr(), a.scales.data_ptr(), a.g.data_ptr(),
                       w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(), M, N, K, a.fmt,
-                      out.data_ptr(), out.stride(0), o, None, 0, _stream()), "fp4_gemm")
+                      out.data_ptr(), out.stride(0), o, None, 0, max_sms, _stream()), "fp4_gemm")
     return out
 
 
-def gemm_plan(M: int, N: int, K: int, fmt: int = NVFP4) -> tuple[int, int, int]:
+def gemm_plan(M: int, N: int, K: int, fmt: int = NVFP4, max_sms: int = 0) -> tuple[int, int, int]:
     """fp4_gemm_plan: (tile_m, tile_n, splits) that fp4_gemm launches."""
     tm, tn, sp = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    _check(L.fp4_gemm_plan(M, N, K, fmt, ctypes.byref(tm), ctypes.byref(tn), ctypes.byref(sp)),
-           "fp4_gemm_plan")
+    _check(L.fp4_gemm_plan(M, N, K, fmt, max_sms, ctypes.byref(tm), ctypes.byref(tn),
+                           ctypes.byref(sp)), "fp4_gemm_plan")
     return tm.value, tn.value, sp.value
 
 

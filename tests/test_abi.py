@@ -53,10 +53,11 @@ def test_scale_bytes_match_oracle_layout(lib, orc):
 def test_gemm_plan_argument_checks(lib):
     i = [ctypes.c_int() for _ in range(3)]
     refs = [ctypes.byref(x) for x in i]
-    assert L.fp4_gemm_plan(8, 256, 100, 0, *refs) == L.FP4_ERR_UNSUPPORTED_SHAPE   # K % 32
-    assert L.fp4_gemm_plan(8, 260, 256, 0, *refs) == L.FP4_ERR_UNSUPPORTED_SHAPE   # N % 8
-    assert L.fp4_gemm_plan(8, 256, 256, 7, *refs) == L.FP4_ERR_INVALID_ARG
-    assert L.fp4_gemm_plan(8, 256, 256, 0, None, refs[1], refs[2]) == L.FP4_ERR_INVALID_ARG
+    assert L.fp4_gemm_plan(8, 256, 100, 0, 0, *refs) == L.FP4_ERR_UNSUPPORTED_SHAPE   # K % 32
+    assert L.fp4_gemm_plan(8, 260, 256, 0, 0, *refs) == L.FP4_ERR_UNSUPPORTED_SHAPE   # N % 8
+    assert L.fp4_gemm_plan(8, 256, 256, 7, 0, *refs) == L.FP4_ERR_INVALID_ARG
+    assert L.fp4_gemm_plan(8, 256, 256, 0, -1, *refs) == L.FP4_ERR_INVALID_ARG       # max_sms
+    assert L.fp4_gemm_plan(8, 256, 256, 0, 0, None, refs[1], refs[2]) == L.FP4_ERR_INVALID_ARG
 
 
 def test_argument_checks_fail_before_any_launch(lib):
@@ -76,14 +77,16 @@ def test_argument_checks_fail_before_any_launch(lib):
     assert q(fake, 4, 256, 0, 0, 0, fake, fake, fake, fake, 16, None) == \
         L.FP4_ERR_WORKSPACE_TOO_SMALL
     g = L.fp4_gemm
-    assert g(fake, fake, fake, fake, fake, fake, 4, 12, 256, 0, fake, 12, 0, None, 0, None) == \
+    assert g(fake, fake, fake, fake, fake, fake, 4, 12, 256, 0, fake, 12, 0, None, 0, 0, None) == \
         L.FP4_ERR_UNSUPPORTED_SHAPE                                   # N % 8
-    assert g(fake, fake, fake, fake, fake, fake, 4, 16, 256, 0, fake, 8, 0, None, 0, None) == \
+    assert g(fake, fake, fake, fake, fake, fake, 4, 16, 256, 0, fake, 8, 0, None, 0, 0, None) == \
         L.FP4_ERR_INVALID_ARG                                         # ldc < N
-    assert g(fake, fake, fake, fake, fake, fake, 4, 16, 256, 0, fake, 20, 0, None, 0, None) == \
+    assert g(fake, fake, fake, fake, fake, fake, 4, 16, 256, 0, fake, 20, 0, None, 0, 0, None) == \
         L.FP4_ERR_MISALIGNED                                          # ldc*2 % 16
-    assert g(fake, fake, None, fake, fake, fake, 4, 16, 256, 0, fake, 16, 0, None, 0, None) == \
+    assert g(fake, fake, None, fake, fake, fake, 4, 16, 256, 0, fake, 16, 0, None, 0, 0, None) == \
         L.FP4_ERR_INVALID_ARG                                         # NVFP4 needs g_a
+    assert g(fake, fake, fake, fake, fake, fake, 4, 16, 256, 0, fake, 16, 0, None, 0, -2, None) == \
+        L.FP4_ERR_INVALID_ARG                                         # max_sms < 0
     f = L.fp4_gemm_fused
     assert f(fake, fake, fake, fake, 33, 16, 256, 0, 0, fake, fake, 16, 0, fake, 1 << 30, None) == \
         L.FP4_ERR_UNSUPPORTED_SHAPE                                   # M > 32

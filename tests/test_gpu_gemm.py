@@ -97,6 +97,28 @@ def test_split_k_is_deterministic(ops, M, N, K, fmt):
     assert all(torch.equal(outs[0], o) for o in outs[1:])
 
 
+@pytest.mark.parametrize("M,N,K,max_sms", [(256, 2880, 2880, 49), (256, 3840, 2880, 37),
+                                           (256, 720, 7680, 37), (2048, 4096, 1024, 40)])
+def test_sm_budget_changes_the_shape_not_the_result(ops, orc, M, N, K, max_sms):
+    """max_sms picks a launch shape for a share of the device (the CTA-pair
+    kernel keeps its tiles and runs fewer persistent pairs); the result
+    stays within tolerance of the oracle (only the FP32 summation order may
+    change)."""
+    if ops.gemm_plan(M, N, K, 0)[0] == 128:
+        assert ops.gemm_plan(M, N, K, 0, max_sms) != ops.gemm_plan(M, N, K, 0)
+    a = inputs.random_bf16(500 + M, (M, K))
+    w = inputs.random_bf16(600 + N, (N, K), 0.02)
+    aq_ref, wq_ref = orc.quantize(a, 0), orc.quantize(w, 0)
+    c_ref = orc.gemm(orc.dequant(aq_ref[0], aq_ref[1], 0, aq_ref[2]),
+                     orc.dequant(wq_ref[0], wq_ref[1], 0, wq_ref[2]))
+    aq = ops.quantize(a.cuda(), 0, ops.SCALES_MMA)
+    wq = ops.quantize_weights(w.cuda(), 0)
+    c = ops.gemm(aq, wq, torch.bfloat16, max_sms=max_sms)
+    torch.cuda.synchronize()
+    ok, worst, where = gemm_close(c, c_ref, torch.bfloat16)
+    assert ok, f"worst err/bound {worst:.3g} at {where}"
+
+
 @pytest.mark.parametrize("M", [1, 8, 32])
 @pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096), (4096, 14336)])
 def test_decode_shapes_fused(ops, orc, M, N, K):
