@@ -159,12 +159,13 @@ fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const flo
  * summation order; the split-K reduction runs in a fixed order, so repeated
  * calls give identical bits.  Requires 1 <= M <= 32 (M == 0 is a no-op;
  * FP4_ERR_UNSUPPORTED_SHAPE above 32).  The workspace (fp4_workspace_bytes)
- * holds the partial maxima and the quantized activation. */
+ * holds the partial maxima and the quantized activation.  max_sms as for
+ * fp4_gemm: the SMs the K split is chosen for (0 = all). */
 fp4_status_t fp4_gemm_fused(const void* a, const uint8_t* w_codes, const uint8_t* w_scales,
                             const float* g_w, int M, int N, int K, fp4_format_t fmt,
                             fp4_global_mode_t gmode, float* g_a,
                             void* C, int ldc, fp4_out_t out,
-                            void* ws, size_t ws_bytes, void* stream);
+                            void* ws, size_t ws_bytes, int max_sms, void* stream);
 
 /* Activation quantization without a workspace argument, for callers that
  * cannot allocate device memory: code running while a stream is captured

@@ -199,11 +199,12 @@ fp4_status_t fp4_gemm_plan(int M, int N, int K, fp4_format_t fmt, int max_sms, i
 fp4_status_t fp4_gemm_fused(const void* x, const uint8_t* w_codes, const uint8_t* w_scales,
                             const float* g_w, int M, int N, int K, fp4_format_t fmt,
                             fp4_global_mode_t gmode, float* g_a, void* C, int ldc, fp4_out_t out,
-                            void* ws, size_t ws_bytes, void* stream) {
+                            void* ws, size_t ws_bytes, int max_sms, void* stream) {
   fp4_status_t st;
   if ((st = check_format(fmt)) != FP4_OK) return st;
   if (out != FP4_OUT_BF16 && out != FP4_OUT_F32) return FP4_ERR_INVALID_ARG;
   if (gmode != FP4_GLOBAL_DYNAMIC && gmode != FP4_GLOBAL_STATIC) return FP4_ERR_INVALID_ARG;
+  if (max_sms < 0) return FP4_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (N % 8 != 0 || M > 32) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (M == 0 || N == 0) return FP4_OK;   // nothing is read or written
@@ -235,6 +236,7 @@ fp4_status_t fp4_gemm_fused(const void* x, const uint8_t* w_codes, const uint8_t
   a.out_f32 = out == FP4_OUT_F32;
   a.ws = ws;
   a.ws_bytes = ws_bytes;
+  a.max_sms = max_sms;
   return from_cuda(fp4::launch_gemm_fused(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -54,7 +54,6 @@ constexpr int DX_STEP = kMaxRows * DBK_BYTES;   // 4 KiB activation codes per st
 constexpr int DXS_STEP = kMaxRows * 16;         // activation scales per step, 16 B per row
 constexpr int kMaxSplits = 8;                // portable cluster size
 constexpr int kThreads = 192;
-constexpr int kTargetCtas = 2 * 148;         // one wave of two CTAs per SM
 // Every CTA reads the whole activation (amax) and quantizes M x its K slice:
 // beyond these sizes the three-kernel chain, which quantizes once, is faster
 // (measured on B200).
@@ -77,7 +76,7 @@ struct DPlan {
 
 // The largest split count S <= 8 whose grid fits one wave of two CTAs per
 // SM; the path applies when every slice then has at most kMaxSteps steps.
-DPlan make_dplan(int M, int N, int K) {
+DPlan make_dplan(int M, int N, int K, int sms) {
   DPlan p{};
   p.n_tiles = (N + DBM - 1) / DBM;
   p.k_steps = (K + DBK - 1) / DBK;
@@ -92,7 +91,7 @@ DPlan make_dplan(int M, int N, int K) {
   const int cap = few_slices ? std::max(4, (p.k_steps + kMaxSteps - 1) / kMaxSteps) : kMaxSplits;
   int s = 1;
   for (int t = 2; t <= kMaxSplits && t <= cap && t <= p.k_steps; ++t)
-    if (p.n_tiles * t <= kTargetCtas) s = t;
+    if (p.n_tiles * t <= 2 * sms) s = t;
   p.splits = s;
   const int slice_steps = (p.k_steps + s - 1) / s;
   p.ok = M >= 1 && M <= kMaxRows && static_cast<long long>(M) * K <= kMaxActValues &&
@@ -492,10 +491,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-bool decode_supported(int M, int N, int K) { return make_dplan(M, N, K).ok; }
+bool decode_supported(int M, int N, int K, int max_sms) {
+  return make_dplan(M, N, K, gemm_sms(max_sms)).ok;
+}
 
 cudaError_t launch_decode(const FusedArgs& f, cudaStream_t s) {
-  const DPlan pl = make_dplan(f.M, f.N, f.K);
+  const DPlan pl = make_dplan(f.M, f.N, f.K, gemm_sms(f.max_sms));
   if (!pl.ok) return cudaErrorInvalidValue;
   DParams p{};
   p.x = static_cast<const uint16_t*>(f.a);

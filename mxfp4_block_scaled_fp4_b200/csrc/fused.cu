@@ -57,7 +57,6 @@ constexpr int FSF_STAGE = 4 * 512;          // up to 4 scale atoms (weights or a
 constexpr int FX_STAGE = 32 * FBK_BYTES;    // activation codes, up to 32 rows
 constexpr int kMaxSplits = 8;               // portable cluster size
 constexpr int kFusedThreads = 192;          // TMA, MMA, 4 worker warps
-constexpr int kTargetCtas = 148;            // SMs of a B200
 constexpr int SMEM_BYTES =
     1024 + FSTAGES * (FW_STAGE + 2 * FSF_STAGE + FX_STAGE) + 256;   // two CTAs fit an SM
 // Tensor-memory columns; every scale-factor address an MMA gets is a
@@ -77,7 +76,7 @@ struct Plan {
 
 // Split count: the largest S <= 8 (one cluster) whose grid fits one wave of
 // two CTAs per SM.
-Plan make_plan(int M, int N, int K, int fmt) {
+Plan make_plan(int M, int N, int K, int fmt, int sms) {
   Plan p{};
   p.n_tiles = (N + FBM - 1) / FBM;
   p.k_steps = (K + FBK - 1) / FBK;
@@ -92,7 +91,7 @@ Plan make_plan(int M, int N, int K, int fmt) {
   const int cap = few_slices ? 4 : kMaxSplits;
   int s = 1;
   for (int t = 2; t <= cap && t <= p.k_steps; ++t)
-    if (p.n_tiles * t <= 2 * kTargetCtas) s = t;
+    if (p.n_tiles * t <= 2 * sms) s = t;
   p.splits = s;
   const int nsf = nsf_of(K, fmt);
   p.off_partial = 0;
@@ -436,12 +435,12 @@ bool make_map(CUtensorMap* m, const uint8_t* base, int rows, int K, int box_rows
 bool fused_supported(int M, int N, int K) { return M >= 1 && M <= 32 && N >= 1 && K >= 1; }
 
 size_t fused_workspace_bytes(int M, int N, int K, int fmt) {
-  return make_plan(M, N, K, fmt).ws_bytes;
+  return make_plan(M, N, K, fmt, 1).ws_bytes;   // (independent of the split)
 }
 
 cudaError_t launch_gemm_fused(const FusedArgs& f, cudaStream_t s) {
-  if (decode_supported(f.M, f.N, f.K)) return launch_decode(f, s);
-  const Plan pl = make_plan(f.M, f.N, f.K, f.fmt);
+  if (decode_supported(f.M, f.N, f.K, f.max_sms)) return launch_decode(f, s);
+  const Plan pl = make_plan(f.M, f.N, f.K, f.fmt, gemm_sms(f.max_sms));
   uint8_t* ws = static_cast<uint8_t*>(f.ws);
   uint8_t* x_codes = ws + pl.off_codes;
   uint8_t* x_scales = ws + pl.off_scales;

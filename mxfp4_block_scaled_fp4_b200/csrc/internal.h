@@ -104,6 +104,7 @@ struct FusedArgs {
   float* g_a;
   void* C; int ldc; int out_f32;
   void* ws; size_t ws_bytes;
+  int max_sms;          // SMs the launch shape is chosen for, 0 = the device's
 };
 size_t fused_workspace_bytes(int M, int N, int K, int fmt);
 // Shapes the fused path takes: 1 <= M <= 32 and K up to 8 slices of 8192.
@@ -111,7 +112,7 @@ bool fused_supported(int M, int N, int K);
 cudaError_t launch_gemm_fused(const FusedArgs& a, cudaStream_t s);
 // The one-kernel path of launch_gemm_fused (M <= 32, M * K <= 128K values,
 // K slices of at most 8 steps of 256).
-bool decode_supported(int M, int N, int K);
+bool decode_supported(int M, int N, int K, int max_sms);
 cudaError_t launch_decode(const FusedArgs& a, cudaStream_t s);
 
 }  // namespace fp4

@@ -123,7 +123,7 @@ class SyntheticDecoder:
         w = self.wq[li][name]
         ws = self._ws(x.shape[0], w.rows, w.K)
         if x.shape[0] <= 32:
-            ops.gemm_fused(x, w, out=out, ws=ws)
+            ops.gemm_fused(x, w, out=out, ws=ws, max_sms=self.max_sms)
         else:
             ops.gemm(ops.quantize(x, self.fmt, ops.SCALES_MMA, ws=ws), w, out=out,
                      max_sms=self.max_sms)

@@ -59,7 +59,7 @@ SIGNATURES = {
     "fp4_quantize_act": (I, [P, I, I, I, I, I, FP, U8P, U8P, P, SZ, P]),
     "fp4_quantize_weights": (I, [P, I, I, I, U8P, U8P, FP, P, SZ, P]),
     "fp4_gemm": (I, [U8P, U8P, FP, U8P, U8P, FP, I, I, I, I, P, I, I, P, SZ, I, P]),
-    "fp4_gemm_fused": (I, [P, U8P, U8P, FP, I, I, I, I, I, FP, P, I, I, P, SZ, P]),
+    "fp4_gemm_fused": (I, [P, U8P, U8P, FP, I, I, I, I, I, FP, P, I, I, P, SZ, I, P]),
     "fp4_gemm_plan": (I, [I, I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
     "fp4_quantize_act_noalloc": (I, [P, I, I, I, I, I, FP, U8P, U8P, P]),
     "fp4_device_status": (I, [ctypes.POINTER(ctypes.c_uint), P]),
@@ -125,9 +125,9 @@ def fp4_gemm(a_codes, a_scales, g_a, w_codes, w_scales, g_w, M, N, K, fmt, C, ld
 
 
 def fp4_gemm_fused(a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc, out, ws,
-                   ws_bytes, stream):
+                   ws_bytes, max_sms, stream):
     return _call("fp4_gemm_fused", a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc,
-                 out, ws, ws_bytes, stream)
+                 out, ws, ws_bytes, max_sms, stream)
 
 
 def fp4_gemm_plan(M, N, K, fmt, max_sms, tile_m, tile_n, splits):

@@ -126,9 +126,11 @@ def gemm_plan(M: int, N: int, K: int, fmt: int = NVFP4, max_sms: int = 0) -> tup
 
 def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
                g_a: torch.Tensor | None = None, out: torch.Tensor | None = None,
-               g_out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
+               g_out: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+               max_sms: int = 0) -> torch.Tensor:
     """fp4_gemm_fused: quantize x (M <= 32) on the fly and multiply with w.
-    ws: as for quantize (concurrent calls need their own)."""
+    ws: as for quantize (concurrent calls need their own); max_sms as for
+    gemm."""
     _cuda_bf16_2d(x, "x")
     M, K = x.shape
     N = w.rows
@@ -147,7 +149,7 @@ def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
     _check(L.fp4_gemm_fused(x.data_ptr(), w.codes.data_ptr(), w.scales.data_ptr(),
                             w.g.data_ptr(), M, N, K, w.fmt, gmode, g_a.data_ptr(),
                             out.data_ptr(), out.stride(0), o, ws.data_ptr(), ws.numel(),
-                            _stream()), "fp4_gemm_fused")
+                            max_sms, _stream()), "fp4_gemm_fused")
     return out
 
 

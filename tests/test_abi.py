@@ -88,10 +88,12 @@ def test_argument_checks_fail_before_any_launch(lib):
     assert g(fake, fake, fake, fake, fake, fake, 4, 16, 256, 0, fake, 16, 0, None, 0, -2, None) == \
         L.FP4_ERR_INVALID_ARG                                         # max_sms < 0
     f = L.fp4_gemm_fused
-    assert f(fake, fake, fake, fake, 33, 16, 256, 0, 0, fake, fake, 16, 0, fake, 1 << 30, None) == \
+    assert f(fake, fake, fake, fake, 33, 16, 256, 0, 0, fake, fake, 16, 0, fake, 1 << 30, 0, None) == \
         L.FP4_ERR_UNSUPPORTED_SHAPE                                   # M > 32
-    assert f(fake, fake, fake, fake, 8, 16, 256, 0, 0, fake, fake, 16, 0, fake, 16, None) == \
+    assert f(fake, fake, fake, fake, 8, 16, 256, 0, 0, fake, fake, 16, 0, fake, 16, 0, None) == \
         L.FP4_ERR_WORKSPACE_TOO_SMALL
+    assert f(fake, fake, fake, fake, 8, 16, 256, 0, 0, fake, fake, 16, 0, fake, 1 << 30, -1, None) == \
+        L.FP4_ERR_INVALID_ARG                                         # max_sms < 0
 
 
 def test_no_gpu_means_no_device_status(lib):
