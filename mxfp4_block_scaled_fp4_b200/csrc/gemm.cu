@@ -41,6 +41,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "launch_shape.h"
 #include "ptx.cuh"
 
 namespace fp4 {
@@ -711,58 +712,6 @@ int max_clusters_bn(int bn, int size) {
                                                          : max_clusters<64>(size);
 }
 
-struct Shape {
-  int bn = 256;     // output tile width
-  int splits = 1;   // CTAs per tile along K
-};
-
-// Tile width and K split for the 128-row kernel, from a time model fitted
-// to B200 measurements of these kernels (graph-launched, back to back): a
-// CTA streams its A and W tiles (128 + BN rows of 144 bytes of codes and
-// scales per K step) at about 112 bytes/ns; a split-K cluster adds about
-// 1.5 us (two cluster barriers, the exchange's latency) plus the
-// (S-1)/S x 128 x BN fp32 partial sums a CTA sends at about 41 bytes/ns
-// (the SM-to-SM rate).  Narrow tiles are only taken when all CTAs fit in
-// one wave; splits only with BN <= 128 and on at most 85% of the SMs (with
-// 256-wide tiles, or clusters on nearly every SM, they measured slower
-// than every alternative).
-Shape choose_shape(int m_tiles, int N, int k_steps, int sms) {
-  Shape best;
-  double best_t = 1e30;
-  for (int bn : {256, 128, 64}) {
-    const int tiles = m_tiles * ((N + bn - 1) / bn);
-    for (int S = 1; S <= 8; ++S) {
-      const int k_per = (k_steps + S - 1) / S;
-      double t;
-      if (S == 1) {
-        if (bn != 256 && tiles > sms) continue;
-        const int waves = (tiles + sms - 1) / sms;
-        t = waves * (128.0 + bn) * k_per * 144.0 / 112.0;
-      } else {
-        if (bn == 256 || (k_steps + k_per - 1) / k_per != S || tiles * S * 100 > sms * 85)
-          continue;
-        if (tiles > max_clusters_bn(bn, S)) continue;
-        t = (128.0 + bn) * k_per * 144.0 / 112.0 + 1500.0 +
-            (S - 1.0) / S * 128.0 * bn * 4.0 / 41.0;
-      }
-      if (t < best_t) {
-        best_t = t;
-        best.bn = bn;
-        best.splits = S;
-      }
-    }
-  }
-  return best;
-}
-
-// The CTA-pair kernel for M > 128 when its 256 x 256 tiles keep at least
-// half the SMs busy; otherwise 128-row tiles, narrower and / or split along
-// K when they are few.
-bool takes_pair(int M, int N, int sms) {
-  const int pair_ctas = 2 * ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256);
-  return M > BM && 2 * pair_ctas >= sms;
-}
-
 template <int BN>
 cudaError_t launch_bn(const GemmArgs& a, Params p, int splits, cudaStream_t s) {
   const int sms = gemm_sms(a.max_sms);
@@ -807,7 +756,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   p.w_rowblocks = (a.N + 127) / 128;
   p.watchdog = watchdog_ptr();
   if (!p.watchdog) return cudaErrorInvalidSymbol;
-  const Shape sh = choose_shape(p.m_tiles, a.N, p.k_steps, sms);
+  const Shape sh = choose_shape(p.m_tiles, a.N, p.k_steps, sms, max_clusters_bn);
   if (sh.bn == 64) return launch_bn<64>(a, p, sh.splits, s);
   if (sh.bn == 128) return launch_bn<128>(a, p, sh.splits, s);
   return launch_bn<256>(a, p, sh.splits, s);
@@ -822,7 +771,7 @@ cudaError_t gemm_plan(int M, int N, int K, int max_sms, int* tile_m, int* tile_n
     *splits = 1;
     return cudaSuccess;
   }
-  const Shape sh = choose_shape((M + BM - 1) / BM, N, (K + BK - 1) / BK, sms);
+  const Shape sh = choose_shape((M + BM - 1) / BM, N, (K + BK - 1) / BK, sms, max_clusters_bn);
   *tile_m = BM;
   *tile_n = sh.bn;
   *splits = sh.splits;
