@@ -36,6 +36,7 @@
 
 #include "codec.cuh"
 #include "internal.h"
+#include "launch_shape.h"
 #include "ptx.cuh"
 
 namespace fp4 {
@@ -81,17 +82,8 @@ DPlan make_dplan(int M, int N, int K, int sms) {
   p.n_tiles = (N + DBM - 1) / DBM;
   p.k_steps = (K + DBK - 1) / DBK;
   p.nmma_n = M <= 16 ? 16 : 32;
-  // K slices, at most one wave of two CTAs per SM.  At M <= 4 with many
-  // weight tiles, up to 4 (further splits add more cluster-reduction cost
-  // than their shorter weight streams save: measured on B200, M=1 4096x4096
-  // 6.7 us with 8 slices, 5.8 us with 4), more only where a slice would
-  // exceed kMaxSteps; with few tiles (M=1 720x7680: 5.7 us with 8 slices,
-  // 7.0 us with 4) or more rows to quantize per slice (M=8), up to 8.
-  const bool few_slices = M <= 4 && p.n_tiles * 4 >= 64;
-  const int cap = few_slices ? std::max(4, (p.k_steps + kMaxSteps - 1) / kMaxSteps) : kMaxSplits;
-  int s = 1;
-  for (int t = 2; t <= kMaxSplits && t <= cap && t <= p.k_steps; ++t)
-    if (p.n_tiles * t <= 2 * sms) s = t;
+  static_assert(kMaxSplits == 8, "decode_splits assumes portable clusters of 8");
+  const int s = decode_splits(M, p.n_tiles, p.k_steps, sms, kMaxSteps);
   p.splits = s;
   const int slice_steps = (p.k_steps + s - 1) / s;
   p.ok = M >= 1 && M <= kMaxRows && static_cast<long long>(M) * K <= kMaxActValues &&

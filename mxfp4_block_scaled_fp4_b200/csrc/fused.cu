@@ -42,6 +42,7 @@
 #include <algorithm>
 
 #include "internal.h"
+#include "launch_shape.h"
 #include "ptx.cuh"
 
 namespace fp4 {
@@ -81,17 +82,8 @@ Plan make_plan(int M, int N, int K, int fmt, int sms) {
   p.n_tiles = (N + FBM - 1) / FBM;
   p.k_steps = (K + FBK - 1) / FBK;
   p.nmma_n = M <= 16 ? 16 : 32;
-  // K slices within one wave: up to 4 when 4 slices still give >= 128 CTAs
-  // and the slices' partial sums are large (M > 16) or their weight streams
-  // long (>= 32 K steps) -- further splits then cost more in cluster
-  // reduction than they save: measured on B200, M=8 4096x14336 18.7 ->
-  // 15.4 us, M=32 4096x4096 13.0 -> 11.9 us; else up to 8 (M=16 4096x4096
-  // 10.0 us with 8 slices, 10.8 with 4; 720x7680 9.3 vs 11.2 us)
-  const bool few_slices = p.n_tiles * 4 >= 128 && (M > 16 || p.k_steps >= 32);
-  const int cap = few_slices ? 4 : kMaxSplits;
-  int s = 1;
-  for (int t = 2; t <= cap && t <= p.k_steps; ++t)
-    if (p.n_tiles * t <= 2 * sms) s = t;
+  static_assert(kMaxSplits == 8, "chain_splits assumes portable clusters of 8");
+  const int s = chain_splits(M, p.n_tiles, p.k_steps, sms);
   p.splits = s;
   const int nsf = nsf_of(K, fmt);
   p.off_partial = 0;

@@ -59,4 +59,41 @@ Shape choose_shape(int m_tiles, int N, int k_steps, int sms, MaxClusters max_clu
   return best;
 }
 
+// K slices of the one-kernel decode path (fp4_gemm_fused, small M): at most
+// one wave of two CTAs per SM on `sms` SMs and at most 8 (a portable
+// cluster).  At M <= 4 with many weight tiles, up to 4 (further splits add
+// more cluster-reduction cost than their shorter weight streams save:
+// measured on B200, M=1 4096x4096 6.7 us with 8 slices, 5.8 us with 4),
+// more only where a slice would exceed max_steps K steps; with few tiles
+// (M=1 720x7680: 5.7 us with 8 slices, 7.0 us with 4) or more rows to
+// quantize per slice (M=8), up to 8.
+inline int decode_splits(int M, int n_tiles, int k_steps, int sms, int max_steps) {
+  int cap = 8;
+  if (M <= 4 && n_tiles * 4 >= 64) {
+    cap = (k_steps + max_steps - 1) / max_steps;   // slices that keep a slice <= max_steps
+    if (cap < 4) cap = 4;
+  }
+  int s = 1;
+  for (int t = 2; t <= 8 && t <= cap && t <= k_steps; ++t)
+    if (n_tiles * t <= 2 * sms) s = t;
+  return s;
+}
+
+// K slices of the small-M chain's GEMM (fp4_gemm_fused above the one-kernel
+// limit), within one wave of two CTAs per SM and at most 8: up to 4 when 4
+// slices still give >= 128 CTAs and the slices' partial sums are large
+// (M > 16) or their weight streams long (>= 32 K steps) -- further splits
+// then cost more in cluster reduction than they save: measured on B200,
+// M=8 4096x14336 18.7 -> 15.4 us, M=32 4096x4096 13.0 -> 11.9 us; else up
+// to 8 (M=16 4096x4096 10.0 us with 8 slices, 10.8 with 4; 720x7680 9.3
+// vs 11.2 us).
+inline int chain_splits(int M, int n_tiles, int k_steps, int sms) {
+  const bool few_slices = n_tiles * 4 >= 128 && (M > 16 || k_steps >= 32);
+  const int cap = few_slices ? 4 : 8;
+  int s = 1;
+  for (int t = 2; t <= cap && t <= k_steps; ++t)
+    if (n_tiles * t <= 2 * sms) s = t;
+  return s;
+}
+
 }  // namespace fp4

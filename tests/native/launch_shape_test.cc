@@ -1,6 +1,7 @@
-// The launch-shape rules of fp4_gemm (csrc/launch_shape.h) on the CPU: the
-// choices for the decoder's M=256 shapes and for SM shares, with a device
-// that can hold as many clusters as SMs allow.  Exit status 0 = all as
+// The launch-shape rules (csrc/launch_shape.h) on the CPU: fp4_gemm's
+// choices for the decoder's M=256 shapes and for SM shares (with a device
+// that can hold as many clusters as SMs allow), and the K slices of
+// fp4_gemm_fused's decode kernel and chain.  Exit status 0 = all as
 // expected (each mismatch is printed).
 #include <cstdio>
 
@@ -28,6 +29,13 @@ void expect_pair(int M, int N, int sms, bool pair) {
   }
 }
 
+void expect_eq(const char* what, int got, int want) {
+  if (got != want) {
+    std::printf("%s: got %d, expected %d\n", what, got, want);
+    ++failures;
+  }
+}
+
 }  // namespace
 
 int main() {
@@ -50,6 +58,22 @@ int main() {
   expect_pair(256, 2880, 148, false);
   expect_pair(128, 28672, 148, false);   // 128 rows: one CTA per tile
   expect_pair(2048, 4096, 40, true);
+  // K slices of the fused small-M path: one-kernel decode (n_tiles = N/128,
+  // K steps of 256, slices of at most 8 steps) and the chain's GEMM
+  expect_eq("decode M=1 4096x4096", fp4::decode_splits(1, 32, 16, 148, 8), 4);
+  expect_eq("decode M=1 2880x2880", fp4::decode_splits(1, 23, 12, 148, 8), 4);
+  expect_eq("decode M=1 720x7680", fp4::decode_splits(1, 6, 30, 148, 8), 8);
+  expect_eq("decode M=1 4096x14336", fp4::decode_splits(1, 32, 56, 148, 8), 7);
+  expect_eq("decode M=1 14336x4096", fp4::decode_splits(1, 112, 16, 148, 8), 2);
+  expect_eq("decode M=8 4096x4096", fp4::decode_splits(8, 32, 16, 148, 8), 8);
+  expect_eq("decode M=1 2880x2880, 49 SMs", fp4::decode_splits(1, 23, 12, 49, 8), 4);
+  expect_eq("decode M=1 2880x2880, 10 SMs", fp4::decode_splits(1, 23, 12, 10, 8), 1);
+  expect_eq("chain M=8 4096x14336", fp4::chain_splits(8, 32, 56, 148), 4);
+  expect_eq("chain M=16 4096x4096", fp4::chain_splits(16, 32, 16, 148), 8);
+  expect_eq("chain M=32 4096x4096", fp4::chain_splits(32, 32, 16, 148), 4);
+  expect_eq("chain M=16 2880x2880", fp4::chain_splits(16, 23, 12, 148), 8);
+  expect_eq("chain M=16 720x7680", fp4::chain_splits(16, 6, 30, 148), 8);
+  expect_eq("chain M=32 14336x4096", fp4::chain_splits(32, 112, 16, 148), 2);
   if (failures == 0) std::printf("launch shapes ok\n");
   return failures == 0 ? 0 : 1;
 }
