@@ -17,7 +17,7 @@
  *        E8M0 power-of-two exponent; NVFP4 = 16-value blocks, E4M3 scale plus
  *        an FP32 per-tensor scale; E2M1 = sign, 2 exponent bits, 1 mantissa.
  *
- * Readings where the pages leave a step open (each is listed in the design doc):
+ * Readings where the pages leave a step open:
  *  R1 every FP32 step below is one correctly rounded IEEE binary32
  *     operation (round to nearest even), no FMA contraction; bf16 inputs are
  *     widened exactly to FP32;
