@@ -62,7 +62,9 @@ typedef enum {
     FP4_ERR_WORKSPACE_TOO_SMALL = 4,
     FP4_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
     FP4_ERR_DEVICE_TIMEOUT = 6,     /* a kernel's bounded wait ran out */
-    FP4_ERR_NO_DEVICE = 7           /* no sm_100 device is current */
+    FP4_ERR_NO_DEVICE = 7,          /* no sm_100 device is current */
+    FP4_ERR_NONFINITE = 8           /* a DYNAMIC amax met an Inf or NaN input
+                                       (reported by fp4_device_status) */
 } fp4_status_t;
 
 typedef enum { FP4_NVFP4 = 0, FP4_MXFP4 = 1 } fp4_format_t;
@@ -167,27 +169,6 @@ fp4_status_t fp4_gemm_fused(const void* a, const uint8_t* w_codes, const uint8_t
                             void* C, int ldc, fp4_out_t out,
                             void* ws, size_t ws_bytes, int max_sms, void* stream);
 
-/* Activation quantization without a workspace argument, for callers that
- * cannot allocate device memory: code running while a stream is captured
- * into a CUDA graph (a cudaMalloc there breaks the capture), engines that
- * reserve all device memory at start-up and allow no later allocation, and
- * latency-critical paths that cannot pay for cudaMalloc's implicit
- * synchronization.  The pages have no counterpart of this entry point.
- * Same arguments (minus ws / ws_bytes), arithmetic and results as
- * fp4_quantize_act.  The DYNAMIC global-scale reduction keeps its partial
- * maxima in a fixed 4 KiB device array inside the library instead of a
- * caller workspace; the array exists on every GPU that loads the library
- * until the process exits.  Limit: the call is rejected with
- * FP4_ERR_WORKSPACE_TOO_SMALL if the scratch it needs
- * (fp4_workspace_bytes(rows, 0, K, fmt)) exceeds those 4 KiB; today that
- * need is 4 KiB for every accepted size.  The first DYNAMIC call on a device
- * looks up the array's device address (cudaGetSymbolAddress, once per
- * device); make that first call before any stream capture.  All calls share
- * the array: calls that overlap on the GPU (other streams, other host
- * threads on the same device) race and must not be issued.  The array keeps
- * the last call's contents; no clearing is needed since every call writes
- * each slot before reading it.  No cudaMalloc / cudaFree or other allocating
- * call is made. */
 /* The launch shape fp4_gemm takes for an M x N x K problem on the current
  * device, for tests and profiling (nothing is launched; the pages have no
  * counterpart).  *tile_m x *tile_n output tiles (256 x 256: the CTA-pair
@@ -201,14 +182,47 @@ fp4_status_t fp4_gemm_fused(const void* a, const uint8_t* w_codes, const uint8_t
 fp4_status_t fp4_gemm_plan(int M, int N, int K, fp4_format_t fmt, int max_sms,
                            int* tile_m, int* tile_n, int* splits);
 
+/* Activation quantization without a workspace argument, for callers that
+ * cannot allocate device memory: engines that reserve all device memory at
+ * start-up for weights and caches and allow no later allocation, plug-ins
+ * that run inside a host framework which owns the allocator and hands them
+ * no scratch, and latency-critical paths that cannot pay for cudaMalloc's
+ * implicit device synchronization.  The pages have no counterpart of this
+ * entry point.
+ * Same arguments (minus ws / ws_bytes), arithmetic and results as
+ * fp4_quantize_act.  The DYNAMIC global-scale reduction keeps its partial
+ * maxima in a fixed 4 KiB device array inside the library instead of a
+ * caller workspace; the array exists on every GPU that loads the library
+ * until the process exits.  Limit: the call is rejected with
+ * FP4_ERR_WORKSPACE_TOO_SMALL if the scratch that fp4_quantize_act needs for
+ * this size (the same rule) exceeds those 4 KiB; today that need is 4 KiB
+ * for every accepted size.  The first DYNAMIC call on a device looks up the
+ * array's device address (cudaGetSymbolAddress, once per device); make that
+ * first call before any stream capture.  All calls share the array: calls
+ * that overlap on the GPU (other streams, other host threads on the same
+ * device) race and must not be issued.  The array keeps the last call's
+ * contents; no clearing is needed since every call writes each slot before
+ * reading it.  No cudaMalloc / cudaFree or other allocating call is made. */
 fp4_status_t fp4_quantize_act_noalloc(const void* x, int rows, int K, fp4_format_t fmt,
                                       fp4_scale_layout_t layout, fp4_global_mode_t gmode,
                                       float* g, uint8_t* codes, uint8_t* scales,
                                       void* stream);
 
-/* Reads and clears the device watchdog word that kernels set when one of
- * their bounded waits runs out.  Synchronizes `stream`.  *code receives the
- * raw word (0 = no timeout).  Returns FP4_ERR_DEVICE_TIMEOUT if it was set. */
+/* Reads and clears, in one atomic exchange on the device, the library's
+ * status word: kernels OR a bit into it when one of their bounded waits runs
+ * out (bits 0-6) and when a DYNAMIC global-scale reduction meets a
+ * non-finite input (bit 7, FP4_STATUS_NONFINITE_BIT).  A bit set by a kernel
+ * on another stream is never lost: it is either returned by this call or
+ * left for the next.  Synchronizes `stream` (the exchange runs on it after
+ * the work queued before).  *code receives the raw word (0 = nothing
+ * happened).  Returns FP4_ERR_DEVICE_TIMEOUT if a wait ran out, else
+ * FP4_ERR_NONFINITE if only the non-finite bit was set, else FP4_OK.
+ * Non-finite inputs are outside the format's contract ("Hardware FP4
+ * inference for speech on Blackwell", section "NVFP4, and the two ways it
+ * fails": the scale saturates, never NaN): the reduction still derives a
+ * finite g from the largest finite bf16 (so no NaN reaches g or alpha), and
+ * the status word reports the input. */
+#define FP4_STATUS_NONFINITE_BIT 0x80u
 fp4_status_t fp4_device_status(unsigned* code, void* stream);
 
 /* Self-test of the failure detection (the pages have no counterpart): one

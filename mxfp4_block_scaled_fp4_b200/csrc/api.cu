@@ -11,8 +11,18 @@
 
 namespace fp4 {
 
-// The watchdog word kernels set when a bounded wait runs out.
+// The status word: kernels OR a bit into it when a bounded wait runs out
+// (the WD_* codes of ptx.cuh) or when a DYNAMIC amax meets a non-finite
+// input (WD_NONFINITE).
 static __device__ unsigned int g_watchdog = 0;
+// Where fp4_device_status's exchange leaves the word it took.
+static __device__ unsigned int g_status_taken = 0;
+
+// Takes the status word and clears it in one atomic exchange, so that a bit
+// a kernel on another stream sets meanwhile is never lost.
+__global__ void status_take_kernel(unsigned* wd, unsigned* taken) {
+  *taken = atomicExch(wd, 0u);
+}
 
 unsigned* watchdog_ptr() {
   static unsigned* cached[64] = {nullptr};
@@ -70,7 +80,7 @@ fp4_status_t device_ok() {
   return cached[dev] == 1 ? FP4_OK : FP4_ERR_NO_DEVICE;
 }
 
-size_t quant_ws_bytes() { return static_cast<size_t>(fp4::kAmaxSlots) * sizeof(unsigned); }
+size_t quant_ws_bytes() { return fp4::quant_workspace_bytes(); }
 
 fp4_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA; }
 
@@ -252,14 +262,22 @@ fp4_status_t fp4_watchdog_selftest(unsigned long long limit_ns, void* stream) {
 
 fp4_status_t fp4_device_status(unsigned* code, void* stream) {
   if (!code) return FP4_ERR_INVALID_ARG;
+  fp4_status_t st;
+  if ((st = device_ok()) != FP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(s) != cudaSuccess) return FP4_ERR_CUDA;
-  unsigned v = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&v, fp4::g_watchdog, sizeof v) != cudaSuccess) return FP4_ERR_CUDA;
-  if (v && cudaMemcpyToSymbol(fp4::g_watchdog, &zero, sizeof zero) != cudaSuccess)
+  unsigned* wd = fp4::watchdog_ptr();
+  void* taken = nullptr;
+  if (!wd || cudaGetSymbolAddress(&taken, fp4::g_status_taken) != cudaSuccess) return FP4_ERR_CUDA;
+  fp4::status_take_kernel<<<1, 1, 0, s>>>(wd, static_cast<unsigned*>(taken));
+  if (cudaGetLastError() != cudaSuccess) return FP4_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, fp4::g_status_taken, sizeof v, 0, cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
     return FP4_ERR_CUDA;
   *code = v;
-  return v ? FP4_ERR_DEVICE_TIMEOUT : FP4_OK;
+  if (v & ~static_cast<unsigned>(fp4::WD_NONFINITE)) return FP4_ERR_DEVICE_TIMEOUT;
+  return v ? FP4_ERR_NONFINITE : FP4_OK;
 }
 
 const char* fp4_status_string(fp4_status_t s) {
@@ -272,6 +290,7 @@ const char* fp4_status_string(fp4_status_t s) {
     case FP4_ERR_CUDA: return "CUDA error";
     case FP4_ERR_DEVICE_TIMEOUT: return "a device-side bounded wait timed out";
     case FP4_ERR_NO_DEVICE: return "no sm_100 device is current";
+    case FP4_ERR_NONFINITE: return "a dynamic global-scale reduction met an Inf or NaN input";
   }
   return "unknown status";
 }

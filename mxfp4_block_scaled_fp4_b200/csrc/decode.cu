@@ -305,6 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) red[warp - 2] = m;
         workers_sync();
         m = max(max(red[0], red[1]), max(red[2], red[3]));
+        // CTA 0 reports a non-finite input; every CTA clamps alike
+        if (m > kBf16MaxFinite)
+          m = (blockIdx.x == 0 && wt == 0) ? amax_checked(m, p.watchdog) : kBf16MaxFinite;
         const float amax = __uint_as_float(m << 16);
         g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
         if (blockIdx.x == 0 && wt == 0) *p.g_a = g;

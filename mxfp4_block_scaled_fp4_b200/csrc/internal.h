@@ -9,6 +9,10 @@ namespace fp4 {
 
 constexpr int kAmaxSlots = 1024;   // partial maxima of the global-scale reduction
 
+// Workspace bytes the activation quantizer needs (the DYNAMIC reduction's
+// partial maxima); one rule for every entry point that quantizes.
+inline size_t quant_workspace_bytes() { return static_cast<size_t>(kAmaxSlots) * sizeof(unsigned); }
+
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count();
 
@@ -53,6 +57,9 @@ struct QuantArgs {
   // DYNAMIC, small tensors: every quantize CTA takes the magnitude maximum
   // of the whole tensor itself (no amax pass, no partial maxima)
   int self_amax = 0;
+  // The status word a non-finite DYNAMIC maximum is reported in (set by
+  // launch_quantize when null).
+  unsigned* status = nullptr;
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl = false);
 

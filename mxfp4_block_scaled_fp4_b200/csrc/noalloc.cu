@@ -1,11 +1,11 @@
 // noalloc.cu -- fp4_quantize_act_noalloc: activation quantization for
 // callers that cannot allocate device memory.
 //
-// Some callers have no way to hand the library a workspace: code that runs
-// while a stream is being captured into a CUDA graph (a cudaMalloc there
-// breaks the capture), engines that reserve all device memory up front for
-// weights and caches and forbid later allocations, and real-time paths that
-// cannot afford cudaMalloc's implicit device synchronization.  This entry
+// Some callers have no way to hand the library a workspace: engines that
+// reserve all device memory up front for weights and caches and forbid
+// later allocations, plug-ins running inside a host framework that owns the
+// allocator and gives them no scratch, and real-time paths that cannot
+// afford cudaMalloc's implicit device synchronization.  This entry
 // point quantizes exactly like fp4_quantize_act, but the scratch that the
 // DYNAMIC global-scale reduction needs (one partial maximum per amax CTA)
 // lives in a fixed file-scope device array instead of a caller workspace.
@@ -30,6 +30,8 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 4096;
 static_assert(kNoAllocScratchBytes >= static_cast<size_t>(kAmaxSlots) * sizeof(unsigned),
               "the scratch must hold every partial maximum of the amax pass");
+// (the size check in the entry point compares quant_workspace_bytes(), the
+// rule fp4_quantize_act applies, with this limit)
 
 // Device-side scratch.  In host code this name is only a host-side stand-in
 // for the symbol, never a device address: its address on a device comes from
@@ -68,9 +70,8 @@ extern "C" fp4_status_t fp4_quantize_act_noalloc(const void* x, int rows, int K,
   if (layout != FP4_SCALES_MMA && layout != FP4_SCALES_ROWMAJOR) return FP4_ERR_INVALID_ARG;
   if (gmode != FP4_GLOBAL_DYNAMIC && gmode != FP4_GLOBAL_STATIC) return FP4_ERR_INVALID_ARG;
   if (rows < 0 || K <= 0 || K % 32 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
-  // the scratch this call needs must fit the fixed array
-  if (fp4_workspace_bytes(rows, 0, K, fmt) > fp4::kNoAllocScratchBytes)
-    return FP4_ERR_WORKSPACE_TOO_SMALL;
+  // the scratch fp4_quantize_act needs (the same rule) must fit the array
+  if (fp4::quant_workspace_bytes() > fp4::kNoAllocScratchBytes) return FP4_ERR_WORKSPACE_TOO_SMALL;
   if (rows == 0) return FP4_OK;
   const bool dyn = fmt == FP4_NVFP4 && gmode == FP4_GLOBAL_DYNAMIC;
   void* scratch = nullptr;

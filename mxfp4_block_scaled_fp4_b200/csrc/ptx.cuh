@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda.h>
 
+#include "fp4.h"
+
 namespace fp4 {
 
 // Watchdog codes: a kernel whose bounded wait runs out ORs one of these into
@@ -17,7 +19,24 @@ enum : unsigned {
   WD_DRAIN    = 1u << 4,   // in-flight copies did not land during unwinding
   WD_STAGING  = 1u << 5,   // scale-staging warps waited too long for a loaded stage
   WD_SELFTEST = 1u << 6,   // the watchdog self-test's wait ran out (expected)
+  WD_NONFINITE = 1u << 7,  // a DYNAMIC amax met an Inf or NaN input (not a wait)
 };
+static_assert(WD_NONFINITE == FP4_STATUS_NONFINITE_BIT, "status bit of fp4.h");
+
+// The largest finite bf16 magnitude pattern.  A magnitude pattern above it
+// is Inf (0x7F80) or NaN.
+constexpr unsigned kBf16MaxFinite = 0x7F7Fu;
+
+// A DYNAMIC global-scale reduction's final maximum (bf16 magnitude bits):
+// a non-finite input is reported in the status word and the maximum is
+// clamped to the largest finite bf16, so g stays finite.
+__device__ __forceinline__ unsigned amax_checked(unsigned m, unsigned* wd) {
+  if (m > kBf16MaxFinite) {
+    atomicOr(wd, WD_NONFINITE);
+    return kBf16MaxFinite;
+  }
+  return m;
+}
 
 // Time budget of one wait (ns).  Legitimate waits here are microseconds.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s

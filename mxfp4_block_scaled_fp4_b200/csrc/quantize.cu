@@ -45,8 +45,11 @@ __device__ __forceinline__ long long mma_scale_offset(long long r, int c, int nc
 // caller's value (STATIC).  g = amax / 2688, 1 for an all-zero tensor.
 // self_amax: the maximum over the whole tensor x (n_vec 16-byte vectors)
 // instead of the partial maxima (small tensors; 4 loads in flight a thread).
+// A non-finite input is reported in `status` and the maximum clamped to the
+// largest finite bf16 (amax_checked), so g stays finite.
 __device__ float global_scale(int dynamic, const float* g, const unsigned* partial,
-                              int n_partial, int self_amax, const uint4* x, long long n_vec) {
+                              int n_partial, int self_amax, const uint4* x, long long n_vec,
+                              unsigned* status) {
   if (!dynamic) return *g;
   __shared__ unsigned red[kThreads / 32];
   unsigned m = 0;
@@ -70,6 +73,9 @@ __device__ float global_scale(int dynamic, const float* g, const unsigned* parti
   __syncthreads();
   m = 0;
   for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) m = max(m, red[i]);
+  // one CTA reports a non-finite input; every CTA clamps alike
+  if (m > kBf16MaxFinite) m = (blockIdx.x == 0 && threadIdx.x == 0) ? amax_checked(m, status)
+                                                                      : kBf16MaxFinite;
   const float amax = __uint_as_float(m << 16);
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
@@ -222,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long
   if (a.release_early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float g = (FMT == 0) ? global_scale(a.dynamic, a.g, a.partial, a.n_partial, a.self_amax,
-                                            static_cast<const uint4*>(a.x), units * 2)
+                                            static_cast<const uint4*>(a.x), units * 2, a.status)
                              : 1.0f;
   if (FMT == 0 && a.dynamic && blockIdx.x == 0 && threadIdx.x == 0) *a.g = g;
   const float six_g = __fmul_rn(6.0f, g);
@@ -319,7 +325,9 @@ QuantGeom quant_geom(const QuantArgs& a) {
 
 }  // namespace
 
-cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl) {
+cudaError_t launch_quantize(const QuantArgs& a_in, cudaStream_t s, bool pdl) {
+  QuantArgs a = a_in;
+  if (!a.status && !(a.status = watchdog_ptr())) return cudaErrorInvalidSymbol;
   const QuantGeom q = quant_geom(a);
   const long long want = std::max((q.units + kThreads * 4 - 1) / (kThreads * 4),
                                   (q.pad_a + q.pad_b + kThreads - 1) / kThreads);

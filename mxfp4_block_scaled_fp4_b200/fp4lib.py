@@ -23,6 +23,9 @@ FP4_ERR_WORKSPACE_TOO_SMALL = 4
 FP4_ERR_CUDA = 5
 FP4_ERR_DEVICE_TIMEOUT = 6
 FP4_ERR_NO_DEVICE = 7
+FP4_ERR_NONFINITE = 8
+# bit of the device status word that reports a non-finite DYNAMIC amax
+FP4_STATUS_NONFINITE_BIT = 0x80
 # fp4_format_t
 FP4_NVFP4 = 0
 FP4_MXFP4 = 1

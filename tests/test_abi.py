@@ -24,7 +24,8 @@ def test_exports_every_header_symbol(lib):
 
 
 def test_status_strings(lib):
-    for s in range(8):
+    for s in range(9):
+        assert L.fp4_status_string(s) != "unknown status"
         assert L.fp4_status_string(s)
     assert L.fp4_status_string(0) == "ok"
     assert L.fp4_status_string(99) == "unknown status"

@@ -126,17 +126,33 @@ def test_decode_shapes_fused(ops, orc, M, N, K):
     run_pair(ops, orc, a, w, 0, "bf16", fused=True)
 
 
-@pytest.mark.parametrize("M,N,K,fmt,dt", [(8192, 28672, 8192, 0, "bf16"),
-                                          (2048, 8192, 8192, 0, "f32"),
-                                          (2048, 8192, 8192, 1, "bf16")])
+# The prefill matrix: M in {2048, 8192} x (N, K) in {(8192, 8192), (28672,
+# 8192)} x {bf16, fp32} in NVFP4, and MXFP4 at both M (bf16).  Cases of one
+# shape are adjacent so that its inputs are generated once.
+PREFILL = [(M, N, 8192, fmt, dt)
+           for M in (2048, 8192) for N in (8192, 28672)
+           for fmt, dt in ((0, "bf16"), (0, "f32"), (1, "bf16"))]
+_prefill_cache = {}
+
+
+def _prefill_inputs(M, N, K):
+    if (M, N, K) not in _prefill_cache:
+        _prefill_cache.clear()
+        _prefill_cache[(M, N, K)] = inputs.prefill(M, N, K)
+    return _prefill_cache[(M, N, K)]
+
+
+@pytest.mark.parametrize("M,N,K,fmt,dt", PREFILL)
 def test_prefill_full_size_sampled(ops, orc, M, N, K, fmt, dt):
     """Full-size launch; the oracle computes 128 sampled rows x 128 sampled
     columns (each row quantized with the tensor's own global scale)."""
-    a, w = inputs.prefill(M, N, K)
+    a, w = _prefill_inputs(M, N, K)
     wq = ops.quantize_weights(w.cuda(), fmt)
     aq = ops.quantize(a.cuda(), fmt, ops.SCALES_MMA)
     c = ops.gemm(aq, wq, DT[dt])
     torch.cuda.synchronize()
+    st, code = ops.device_status()
+    assert st == 0 and code == 0
     rng = np.random.default_rng(M + N)
     ri = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 126, replace=False)]))
     ci = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 126, replace=False)]))
@@ -149,9 +165,11 @@ def test_prefill_full_size_sampled(ops, orc, M, N, K, fmt, dt):
     ca, sa, ga = orc.quantize(a[rt].contiguous(), fmt, g_a)
     cw, sw, gw = orc.quantize(w[ct].contiguous(), fmt, g_w)
     assert np.array_equal(bits(aq.codes[rt.cuda()]), ca)
+    assert np.array_equal(bits(wq.codes[ct.cuda()]), cw)
     c_ref = orc.gemm(orc.dequant(ca, sa, fmt, ga), orc.dequant(cw, sw, fmt, gw))
     ok, worst, where = gemm_close(c[rt.cuda()][:, ct.cuda()], c_ref, DT[dt])
     assert ok, f"worst err/bound {worst:.3g} at {where}"
+    del c, aq, wq
 
 
 # M * K <= 128K values take the one-kernel path, larger activations the
