@@ -5,7 +5,9 @@ TEST INFRASTRUCTURE ONLY.  Only tests/, ``__graft_entry__.smoke()`` and
 this package.  The product library never calls it and shares no code with it.
 
 The arithmetic lives in ``fp4_oracle.c`` (plain C, one correctly rounded
-binary32 operation per step, see the readings R1-R6 in its header).  This
+binary32 operation per step, see the readings R1-R8 in its header: R7 is
+the online Walsh-Hadamard rotation, R8 the overflow-aware MXFP4 scale
+rule).  This
 module marshals numpy arrays and adds the GEMM on dequantized values in
 binary64, which is the plain definition C = A_hat . W_hat^T.
 
@@ -13,7 +15,10 @@ Sources: "Hardware FP4 inference for speech on Blackwell", section "NVFP4,
 and the two ways it fails" (format, scale rule, saturation); "FP4 n'existe
 pas : il existe des FP4, et chaque runtime choisit son dialecte", section
 "Deux dialectes, deux strategies de scaling" (MXFP4 = OCP MX: 32-blocks,
-E8M0 scales).
+E8M0 scales) and section "L'ecart de qualite -- et comment il se reduit"
+(OAS); "FP4 on a consumer RTX 5090: the Blackwell headline loses to plain
+int4", section "Finding 3 -- the real-FP4 path (QuTLASS MXFP4)" (online
+Hadamard rotation ahead of the activation quantizer).
 """
 from __future__ import annotations
 
@@ -74,6 +79,14 @@ def _declare(L):
     L.orc_scales_to_mma.argtypes = [P, i64, i64, P]
     L.orc_scales_from_mma.restype = None
     L.orc_scales_from_mma.argtypes = [P, i64, i64, P]
+    L.orc_amax_f32.restype = ctypes.c_float
+    L.orc_amax_f32.argtypes = [P, i64]
+    L.orc_nvfp4_quantize_f32.restype = ctypes.c_int
+    L.orc_nvfp4_quantize_f32.argtypes = [P, i64, i64, ctypes.c_int, P, P, P]
+    L.orc_mxfp4_quantize_f32.restype = ctypes.c_int
+    L.orc_mxfp4_quantize_f32.argtypes = [P, i64, i64, ctypes.c_int, P, P]
+    L.orc_hadamard_f32.restype = ctypes.c_int
+    L.orc_hadamard_f32.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, P]
     L.orc_e2m1_encode_array.restype = None
     L.orc_e2m1_encode_array.argtypes = [P, i64, P]
     L.orc_e4m3_encode_array.restype = None
@@ -192,6 +205,80 @@ def quantize(x, fmt: int, g: float | None = None):
         return quantize_nvfp4(x, g)
     c, s = quantize_mxfp4(x)
     return c, s, 1.0
+
+
+# ------------------------------------- binary32 inputs, rotation, OAS (R7, R8) --
+
+OCP = 0     # MXFP4 scale rule R5: e = floor(log2 amax) - 2
+OAS = 1     # MXFP4 scale rule R8: the smallest e with amax <= 6 * 2^e
+
+
+def widen_bf16(x) -> np.ndarray:
+    """bf16 bit patterns -> binary32 values (exact: bf16 is the top half)."""
+    x = _as_bf16_bits(x)
+    return (x.astype(np.uint32) << 16).view(np.float32)
+
+
+def rotation_shifts(n: int) -> tuple[int, int]:
+    """(activation shift, weight shift) of R7: they add up to log2(n), so the
+    product of a rotated activation and a rotated weight equals the plain
+    product."""
+    lg = int(n).bit_length() - 1
+    return (lg + 1) // 2, lg // 2
+
+
+def hadamard(x, n: int, shift: int) -> np.ndarray:
+    """R7: every n-value block of every row rotated by the order-n
+    Walsh-Hadamard matrix in binary32 (fast transform), times 2^-shift."""
+    x = _as_bf16_bits(x)
+    rows, K = x.shape
+    out = np.empty((rows, K), np.float32)
+    rc = lib().orc_hadamard_f32(_ptr(x), rows, K, int(n), int(shift), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"bad rotation arguments: shape {x.shape}, n={n}, shift={shift}")
+    return out
+
+
+def amax_f32(x: np.ndarray) -> float:
+    x = np.ascontiguousarray(x, np.float32)
+    return float(lib().orc_amax_f32(_ptr(x), x.size))
+
+
+def quantize_f32(x: np.ndarray, fmt: int, g: float | None = None, rule: int = OCP):
+    """Quantize binary32 values [rows, K] (R1-R5 on binary32 inputs; MXFP4
+    with scale rule `rule`).  Returns (codes, row-major scales, g)."""
+    x = np.ascontiguousarray(x, np.float32)
+    rows, K = x.shape
+    codes = np.empty((rows, K // 2), np.uint8)
+    if fmt == NVFP4:
+        scales = np.empty((rows, K // 16), np.uint8)
+        gbuf = np.array([1.0 if g is None else g], np.float32)
+        rc = lib().orc_nvfp4_quantize_f32(_ptr(x), rows, K, int(g is None), _ptr(gbuf),
+                                          _ptr(codes), _ptr(scales))
+        gv = float(gbuf[0])
+    else:
+        scales = np.empty((rows, K // 32), np.uint8)
+        rc = lib().orc_mxfp4_quantize_f32(_ptr(x), rows, K, int(rule), _ptr(codes),
+                                          _ptr(scales))
+        gv = 1.0
+    if rc != 0:
+        raise ValueError(f"bad shape or rule: {x.shape}, rule {rule}")
+    return codes, scales, gv
+
+
+def quantize_ex(x, fmt: int, g: float | None = None, hadamard_n: int = 0,
+                operand: str = "act", rule: int = OCP):
+    """The quantizer with its options: an online rotation of order
+    hadamard_n (0 = none; the operand's R7 shift) and, for MXFP4, the scale
+    rule.  Without options it is ``quantize``."""
+    if hadamard_n:
+        sa, sw = rotation_shifts(hadamard_n)
+        xf = hadamard(x, hadamard_n, sa if operand == "act" else sw)
+    elif fmt == MXFP4 and rule != OCP:
+        xf = widen_bf16(x).reshape(np.shape(x))
+    else:
+        return quantize(x, fmt, g)
+    return quantize_f32(xf, fmt, g, rule)
 
 
 def dequant(codes: np.ndarray, scales: np.ndarray, fmt: int, g: float = 1.0):

@@ -16,6 +16,10 @@
  *        its format table: MXFP4 = OCP MX v1.0, 32-value blocks sharing an
  *        E8M0 power-of-two exponent; NVFP4 = 16-value blocks, E4M3 scale plus
  *        an FP32 per-tensor scale; E2M1 = sign, 2 exponent bits, 1 mantissa.
+ *  [5090] "FP4 on a consumer RTX 5090: the Blackwell headline loses to plain
+ *        int4", section "Finding 3 -- the real-FP4 path (QuTLASS MXFP4)":
+ *        every layer pays an online Hadamard rotation plus activation
+ *        quantization.
  *
  * Readings where the pages leave a step open:
  *  R1 every FP32 step below is one correctly rounded IEEE binary32
@@ -31,6 +35,26 @@
  *     clamped to [-127, 127], e = -127 when b == 0; scale byte = e + 127;
  *     v = x * 2^-e computed exactly; q = E2M1 RNE with saturation to 6;
  *  R6 packing: element 2j goes to the low nibble of byte j of its row.
+ *  R7 online rotation ([5090], section "Finding 3 -- the real-FP4 path
+ *     (QuTLASS MXFP4)": an online Hadamard rotation ahead of the activation
+ *     quantizer): block-diagonal Walsh-Hadamard along K, n in {16, 32}
+ *     consecutive values per block from k = 0, Sylvester order
+ *     H[i][j] = (-1)^popcount(i & j).  Computed in binary32 as the fast
+ *     transform: for h = 1, 2, 4, ... < n, every pair (i, i + h) with bit h
+ *     of i clear becomes (RN(a + b), RN(a - b)); then every value is
+ *     multiplied by 2^-shift (exact: every intermediate is a multiple of the
+ *     smallest bf16 step, so the scaling never rounds).  The two operands of
+ *     a GEMM take shifts that add up to log2(n), so that the rotated
+ *     product equals the plain one: activations ceil(log2(n)/2), weights
+ *     floor(log2(n)/2).  The quantizers then take the binary32 rotated
+ *     values exactly as they take widened bf16 values (R1-R5), the DYNAMIC
+ *     amax included;
+ *  R8 MXFP4 "overflow-aware" scale rule (OAS; [DIA], section "L'ecart de
+ *     qualite -- et comment il se reduit": the block scale is chosen so
+ *     that the extreme values do not saturate): e = the smallest integer
+ *     with b <= 6 * 2^e, i.e. e = floor(log2 b) - 2 when b / 2^floor(log2 b)
+ *     <= 1.5 and one more otherwise, clamped to [-127, 127] (-127 for a zero
+ *     block).  R5 is the OCP rule, which lets values in (6, 8) * 2^e clip.
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC
  * (oracle/build.py).  FP32 arithmetic is SSE binary32 on x86-64
@@ -169,13 +193,14 @@ float orc_nvfp4_global_scale(float amax)
 
 /* ----------------------------------------------------------- NVFP4 -- */
 
-/* One NVFP4 block of 16 values ([HW4] with R3/R4).  Writes 16 codes
- * (one per byte, unpacked) and returns the E4M3 scale byte. */
-static unsigned nvfp4_block(const uint16_t* x, float g, unsigned char q[16])
+/* One NVFP4 block of 16 binary32 values ([HW4] with R3/R4; bf16 inputs are
+ * widened exactly first).  Writes 16 codes (one per byte, unpacked) and
+ * returns the E4M3 scale byte. */
+static unsigned nvfp4_block(const float* x, float g, unsigned char q[16])
 {
     float b = 0.0f;
     for (int i = 0; i < 16; ++i) {
-        float a = fabsf(orc_bf16_to_f32(x[i]));
+        float a = fabsf(x[i]);
         if (a > b) b = a;
     }
     float d = 6.0f * g;
@@ -189,10 +214,43 @@ static unsigned nvfp4_block(const uint16_t* x, float g, unsigned char q[16])
     float sg = sv * g;
     float r = 1.0f / sg;
     for (int i = 0; i < 16; ++i) {
-        float v = orc_bf16_to_f32(x[i]) * r;
+        float v = x[i] * r;
         q[i] = (unsigned char)orc_e2m1_encode((double)v);
     }
     return s;
+}
+
+/* amax over a binary32 tensor (exact). */
+float orc_amax_f32(const float* x, long n)
+{
+    float m = 0.0f;
+    for (long i = 0; i < n; ++i) {
+        float a = fabsf(x[i]);
+        if (a > m) m = a;
+    }
+    return m;
+}
+
+/* NVFP4 of a row-major binary32 [rows, K] tensor; g as for the bf16 form. */
+int orc_nvfp4_quantize_f32(const float* x, long rows, long K, int dynamic,
+                           float* g, uint8_t* codes, uint8_t* scales)
+{
+    if (rows < 0 || K <= 0 || K % 16 != 0) return ORC_BAD_SHAPE;
+    if (dynamic) *g = orc_nvfp4_global_scale(orc_amax_f32(x, rows * K));
+    const float gg = *g;
+    const long nb = K / 16;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        for (long b = 0; b < nb; ++b) {
+            unsigned char q[16];
+            scales[r * nb + b] =
+                (uint8_t)nvfp4_block(x + r * K + b * 16, gg, q);
+            for (int j = 0; j < 8; ++j)
+                codes[r * (K / 2) + b * 8 + j] =
+                    (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+        }
+    }
+    return ORC_OK;
 }
 
 /* Quantize a row-major bf16 [rows, K] tensor to NVFP4.
@@ -210,9 +268,11 @@ int orc_nvfp4_quantize(const uint16_t* x, long rows, long K, int dynamic,
 #pragma omp parallel for schedule(static)
     for (long r = 0; r < rows; ++r) {
         for (long b = 0; b < nb; ++b) {
+            float xf[16];
             unsigned char q[16];
-            scales[r * nb + b] =
-                (uint8_t)nvfp4_block(x + r * K + b * 16, gg, q);
+            for (int i = 0; i < 16; ++i)
+                xf[i] = orc_bf16_to_f32(x[r * K + b * 16 + i]);
+            scales[r * nb + b] = (uint8_t)nvfp4_block(xf, gg, q);
             for (int j = 0; j < 8; ++j)
                 codes[r * (K / 2) + b * 8 + j] =
                     (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
@@ -236,26 +296,59 @@ static int floor_log2_f32(float a)
     return msb - 149;
 }
 
-/* One MXFP4 block of 32 values (R5).  Returns the E8M0 scale byte. */
-static unsigned mxfp4_block(const uint16_t* x, unsigned char q[32])
+/* The MXFP4 block exponent of a block maximum b >= 0: rule 0 is R5 (OCP,
+ * floor(log2 b) - 2), rule 1 is R8 (OAS: the smallest e with b <= 6 * 2^e).
+ * Clamped to [-127, 127]; -127 for b == 0. */
+static int mxfp4_exponent(float b, int rule)
+{
+    if (b == 0.0f) return -127;
+    int e = floor_log2_f32(b) - 2;
+    if (rule == 1 && (double)b > ldexp(6.0, e)) e += 1;   /* exact comparison */
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* One MXFP4 block of 32 binary32 values (R5 / R8).  Returns the E8M0 scale
+ * byte. */
+static unsigned mxfp4_block(const float* x, int rule, unsigned char q[32])
 {
     float b = 0.0f;
     for (int i = 0; i < 32; ++i) {
-        float a = fabsf(orc_bf16_to_f32(x[i]));
+        float a = fabsf(x[i]);
         if (a > b) b = a;
     }
-    int e = (b == 0.0f) ? -127 : floor_log2_f32(b) - 2;
-    if (e < -127) e = -127;
-    if (e > 127) e = 127;
+    int e = mxfp4_exponent(b, rule);
     for (int i = 0; i < 32; ++i) {
-        double v = ldexp((double)orc_bf16_to_f32(x[i]), -e);   /* exact */
+        double v = ldexp((double)x[i], -e);   /* exact */
         q[i] = (unsigned char)orc_e2m1_encode(v);
     }
     return (unsigned)(e + 127);
 }
 
-/* Quantize a row-major bf16 [rows, K] tensor to MXFP4 (no global scale).
- * codes: [rows, K/2]; scales: [rows, K/32] E8M0 bytes, row-major. */
+/* MXFP4 of a row-major binary32 [rows, K] tensor with scale rule `rule`
+ * (0 = OCP R5, 1 = OAS R8). */
+int orc_mxfp4_quantize_f32(const float* x, long rows, long K, int rule,
+                           uint8_t* codes, uint8_t* scales)
+{
+    if (rows < 0 || K <= 0 || K % 32 != 0 || rule < 0 || rule > 1) return ORC_BAD_SHAPE;
+    const long nb = K / 32;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        for (long b = 0; b < nb; ++b) {
+            unsigned char q[32];
+            scales[r * nb + b] = (uint8_t)mxfp4_block(x + r * K + b * 32, rule, q);
+            for (int j = 0; j < 16; ++j)
+                codes[r * (K / 2) + b * 16 + j] =
+                    (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+        }
+    }
+    return ORC_OK;
+}
+
+/* Quantize a row-major bf16 [rows, K] tensor to MXFP4 (no global scale),
+ * OCP rule (R5).  codes: [rows, K/2]; scales: [rows, K/32] E8M0 bytes,
+ * row-major. */
 int orc_mxfp4_quantize(const uint16_t* x, long rows, long K,
                        uint8_t* codes, uint8_t* scales)
 {
@@ -264,11 +357,45 @@ int orc_mxfp4_quantize(const uint16_t* x, long rows, long K,
 #pragma omp parallel for schedule(static)
     for (long r = 0; r < rows; ++r) {
         for (long b = 0; b < nb; ++b) {
+            float xf[32];
             unsigned char q[32];
-            scales[r * nb + b] = (uint8_t)mxfp4_block(x + r * K + b * 32, q);
+            for (int i = 0; i < 32; ++i)
+                xf[i] = orc_bf16_to_f32(x[r * K + b * 32 + i]);
+            scales[r * nb + b] = (uint8_t)mxfp4_block(xf, 0, q);
             for (int j = 0; j < 16; ++j)
                 codes[r * (K / 2) + b * 16 + j] =
                     (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------- online rotation (R7) -- */
+
+/* Rotate every n-value block of every row of a bf16 [rows, K] tensor by the
+ * Walsh-Hadamard matrix of order n (n = 16 or 32, K % n == 0), in binary32
+ * by the fast transform of R7, then scale by 2^-shift (0 <= shift <= 8).
+ * out: binary32 [rows, K]. */
+int orc_hadamard_f32(const uint16_t* x, long rows, long K, int n, int shift,
+                     float* out)
+{
+    if (rows < 0 || K <= 0 || (n != 16 && n != 32) || K % n != 0 ||
+        shift < 0 || shift > 8)
+        return ORC_BAD_SHAPE;
+    const float scale = ldexpf(1.0f, -shift);
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        for (long b = 0; b < K / n; ++b) {
+            float v[32];
+            for (int i = 0; i < n; ++i) v[i] = orc_bf16_to_f32(x[r * K + b * n + i]);
+            for (int h = 1; h < n; h *= 2)
+                for (int i = 0; i < n; ++i)
+                    if ((i & h) == 0) {
+                        float a = v[i], c = v[i + h];
+                        v[i] = a + c;
+                        v[i + h] = a - c;
+                    }
+            for (int i = 0; i < n; ++i) out[r * K + b * n + i] = v[i] * scale;
         }
     }
     return ORC_OK;
