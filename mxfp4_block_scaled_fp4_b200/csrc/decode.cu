@@ -196,6 +196,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < n_steps; ++i) {
         const int stage = i % DSTAGES;
         const uint32_t phase = static_cast<uint32_t>(i / DSTAGES) & 1u;
+        if (i == DSTAGES) {
+          // the ring is full and frees only once the MMAs run (after the
+          // activation's amax and quantization): the slice's remaining
+          // weight tiles and scale atoms stream into L2 meanwhile
+          for (int j = DSTAGES; j < n_steps; ++j) {
+            const int ksj = s_lo + j, cbj = ksj * kAtoms;
+            tma_prefetch_l2_2d(&tm_w, ksj * DBK_BYTES, tile * DBM);
+            bulk_prefetch_l2(p.w_scales + (static_cast<long long>(tile) * p.ncb + cbj) * 512,
+                             static_cast<uint32_t>(min(kAtoms, p.ncb - cbj)) * 512u);
+          }
+        }
         if (i >= DSTAGES &&
             !mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.watchdog, WD_PRODUCER))
           break;

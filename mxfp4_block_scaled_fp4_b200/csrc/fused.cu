@@ -215,6 +215,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         if (i == first - 1) {
+          // the ring is full and frees only as the MMAs consume it: the
+          // slice's remaining weight tiles and scale atoms stream into L2
+          // while the preceding kernels finish and the ring drains
+          for (int j = first; j < n_steps; ++j) {
+            const int ksj = s_lo + j, cbj = ksj * kAtoms;
+            tma_prefetch_l2_2d(&tm_w, ksj * FBK_BYTES, tile * FBM);
+            bulk_prefetch_l2(p.w_scales + (static_cast<long long>(tile) * p.ncb + cbj) * 512,
+                             static_cast<uint32_t>(min(kAtoms, p.ncb - cbj)) * 512u);
+          }
           // the quantized activation is produced by the preceding kernel
           grid_dep_wait();
           for (int j = 0; j < first; ++j) {
