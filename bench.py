@@ -499,10 +499,125 @@ def measure_prefill_matrix(torch, L, ops, a_big, w_big, dev, fp4_peak):
     return rows
 
 
+MOE_CONFIGS = [(8, 16384, 4096, 4096), (64, 16384, 2048, 4096)]
+
+
+def measure_grouped(torch, ops, dev, fp4_peak):
+    """The grouped (mixture-of-experts) GEMM, fp4_gemm_grouped: E experts of
+    [N, K], 16384 routed rows (8192 tokens x 2 experts each) spread over the
+    experts with Dirichlet(1) proportions (seed 11; uneven groups that start
+    on any row), NVFP4 and MXFP4, bf16 out.  Each call after an L2 flush,
+    median of 20.  Also the same work as E separate fp4_gemm calls."""
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    rows = []
+    for (E, M, N, Kx) in MOE_CONFIGS:
+        rng = np.random.default_rng(11)
+        sizes = np.floor(rng.dirichlet(np.ones(E)) * M).astype(np.int64)
+        sizes[0] += M - sizes.sum()
+        offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(12)
+        a = torch.randn((M, Kx), generator=gen, device=dev).to(torch.bfloat16)
+        w = (torch.randn((E, N, Kx), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+        offs_d = torch.from_numpy(offs).to(dev)
+        flop = 2.0 * M * N * Kx
+        for fmt in (0, 1):
+            aq = ops.quantize(a, fmt, ops.SCALES_MMA)
+            wq = ops.quantize_experts(w, fmt)
+            c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            subs = []
+            for e in range(E):
+                lo, hi = int(offs[e]), int(offs[e + 1])
+                if hi > lo:
+                    subs.append((lo, hi, ops.quantize(a[lo:hi].contiguous(), fmt, ops.SCALES_MMA,
+                                                      g=aq.g if fmt == 0 else None),
+                                 ops.Quantized(wq.codes[e], wq.scales[e], wq.g[e:e + 1], fmt,
+                                               ops.SCALES_MMA, N, Kx)))
+
+            def grouped():
+                ops.gemm_grouped(aq, wq, offs_d, out=c)
+
+            def separate():
+                for lo, hi, sq, one in subs:
+                    ops.gemm(sq, one, out=c[lo:hi])
+
+            res = {}
+            for name, fn in (("grouped", grouped), ("separate_calls", separate)):
+                for _ in range(3):
+                    fn()
+                ts = []
+                for _ in range(20):
+                    flush_l2(torch, flush, flush_r)
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    fn()
+                    e1.record()
+                    torch.cuda.synchronize(dev)
+                    ts.append(e0.elapsed_time(e1))
+                res[name] = float(np.median(ts))
+            rows.append({"E": E, "M_routed": M, "N": N, "K": Kx,
+                         "format": "NVFP4" if fmt == 0 else "MXFP4",
+                         "group_rows_min_max": [int(sizes.min()), int(sizes.max())],
+                         "grouped_ms": round(res["grouped"], 4),
+                         "grouped_tflops": round(flop / res["grouped"] / 1e9, 1),
+                         "grouped_frac_fp4_peak": round(flop / res["grouped"] / 1e9 / fp4_peak, 4),
+                         "separate_calls_ms": round(res["separate_calls"], 4),
+                         "kernel": "fp4 gemm_kernel grouped (128x128 tiles, device-side offsets)"})
+    st, code = ops.device_status()
+    if st != 0:
+        raise RuntimeError(f"status word set in the grouped GEMM: {code:#x}")
+    return rows
+
+
+def measure_gemm_quant(torch, ops, a, w_dev, dev, fp4_peak):
+    """The GEMM whose epilogue emits the next layer's FP4 activation
+    (fp4_gemm_quant, NVFP4 STATIC g and MXFP4) on the prefill matrix's
+    largest shape, against fp4_gemm with bf16 out; each call after an L2
+    flush, median of 20."""
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    Mq, Nq = a.shape[0], w_dev.shape[0]
+    flop = 2.0 * Mq * Nq * K
+    rows = []
+    for fmt in (0, 1):
+        aq = ops.quantize(a, fmt, ops.SCALES_MMA)
+        wq = ops.quantize_weights(w_dev, fmt)
+        g_out = torch.tensor([0.004], dtype=torch.float32, device=dev)
+        c = torch.empty((Mq, Nq), dtype=torch.bfloat16, device=dev)
+        res = {}
+        for name, fn in (("bf16_out", lambda: ops.gemm(aq, wq, out=c)),
+                         ("fp4_out", lambda: ops.gemm_quant(aq, wq, fmt, ops.SCALES_MMA, g_out))):
+            for _ in range(3):
+                fn()
+            ts = []
+            for _ in range(20):
+                flush_l2(torch, flush, flush_r)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1))
+            res[name] = float(np.median(ts))
+        out_bytes = Mq * Nq // 2 + Mq * Nq // (16 if fmt == 0 else 32)
+        rows.append({"M": Mq, "N": Nq, "K": K, "format": "NVFP4" if fmt == 0 else "MXFP4",
+                     "fp4_out_ms": round(res["fp4_out"], 4),
+                     "fp4_out_tflops": round(flop / res["fp4_out"] / 1e9, 1),
+                     "fp4_out_frac_fp4_peak": round(flop / res["fp4_out"] / 1e9 / fp4_peak, 4),
+                     "bf16_out_ms": round(res["bf16_out"], 4),
+                     "bytes_written_fp4_vs_bf16": [out_bytes, Mq * Nq * 2]})
+    return rows
+
+
 def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak):
-    """fp4_quantize_act on the activation-quantize sweep, L2 flushed before
-    every call.  Reports GB/s with single-pass bytes (2.5625 B/elem NVFP4,
-    2.53125 MXFP4) and, for the DYNAMIC NVFP4 run, with both reads of the
+    """fp4_quantize_act_ex on the activation-quantize sweep, L2 flushed
+    before every call: NVFP4 DYNAMIC / STATIC, MXFP4, and the options (the
+    online Hadamard rotation of order 16 / 32, the overflow-aware MXFP4
+    rule).  Reports GB/s with single-pass bytes (2.5625 B/elem NVFP4,
+    2.53125 MXFP4) and, for the DYNAMIC NVFP4 runs, with both reads of the
     amax pass (4.5625 B/elem)."""
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
@@ -510,7 +625,11 @@ def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak):
     res = []
     for (M, K) in SWEEP_SHAPES:
         x = inputs.act_sweep(M, K).to(dev)
-        for fmt, gmode, name in ((0, 0, "nvfp4_dynamic"), (0, 1, "nvfp4_static"), (1, 0, "mxfp4")):
+        for fmt, gmode, name, had, rule in (
+                (0, 0, "nvfp4_dynamic", 0, 0), (0, 1, "nvfp4_static", 0, 0), (1, 0, "mxfp4", 0, 0),
+                (0, 0, "nvfp4_dynamic_hadamard16", 16, 0), (1, 0, "mxfp4_hadamard32", 32, 0),
+                (1, 0, "mxfp4_oas", 0, 1)):
+            opt = L.opts(had, rule)
             codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
             scales = torch.empty(L.fp4_scale_bytes(M, K, fmt, 0), dtype=torch.uint8, device=dev)
             g = torch.full((1,), 0.05, dtype=torch.float32, device=dev)
@@ -522,8 +641,9 @@ def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak):
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record()
-                st = L.fp4_quantize_act(x.data_ptr(), M, K, fmt, 0, gmode, g.data_ptr(),
-                                        codes.data_ptr(), scales.data_ptr(), ws.data_ptr(), wsb, sp)
+                st = L.fp4_quantize_act_ex(x.data_ptr(), M, K, fmt, 0, gmode, opt, g.data_ptr(),
+                                           codes.data_ptr(), scales.data_ptr(), ws.data_ptr(),
+                                           wsb, sp)
                 e1.record()
                 torch.cuda.synchronize(dev)
                 assert st == 0
@@ -605,6 +725,9 @@ def run_part(args, rank):
         line["decode"] = measure_decode(torch, ops, L, inputs, dev, peaks["hbm_gbs"], shapes)
     elif args.only == "decoder":
         line["decoder"] = measure_decoder(torch, dev)
+    elif args.only == "grouped":
+        peaks_fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16
+        line["grouped"] = measure_grouped(torch, ops, dev, peaks_fp4)
     else:
         line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"])
     if rank == 0:
@@ -641,7 +764,7 @@ def main():
     ap.add_argument("--no-suite", action="store_true",
                     help="skip the decode and quantize-sweep measurements")
     ap.add_argument("--only", default="all",
-                    choices=["all", "prefill", "decode", "quantize", "decoder"],
+                    choices=["all", "prefill", "decode", "quantize", "decoder", "grouped"],
                     help="run one part only (profiling); the JSON line then carries that part")
     ap.add_argument("--decode-shape", default=None, help="M,N,K: restrict the decode part")
     ap.add_argument("--shape", default=None,
@@ -658,7 +781,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank)
-    if args.only in ("decode", "quantize", "decoder"):
+    if args.only in ("decode", "quantize", "decoder", "grouped"):
         return run_part(args, rank)
     if args.warmup < 3:
         args.warmup = 3
@@ -849,6 +972,8 @@ def main():
     }
     if not args.no_suite and (M, N, K) == (8192, 28672, 8192):
         line["prefill_matrix"] = measure_prefill_matrix(torch, L, ops, a, w_dev, dev, fp4_peak)
+        line["gemm_quant"] = measure_gemm_quant(torch, ops, a, w_dev, dev, fp4_peak)
+        line["grouped"] = measure_grouped(torch, ops, dev, fp4_peak)
     if not args.no_suite:
         line["decode"] = measure_decode(torch, ops, L, inputs, dev, peaks["hbm_gbs"])
         line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"])

@@ -109,6 +109,45 @@ fp4_status_t fp4_quantize_act(const void* x, int rows, int K, fp4_format_t fmt,
                               float* g, uint8_t* codes, uint8_t* scales,
                               void* ws, size_t ws_bytes, void* stream);
 
+/* Options of the extended quantizer entry points below.  Passing NULL, or a
+ * zeroed struct, gives exactly the plain entry points' results.
+ *  hadamard  0: none.  16 or 32: an online rotation of every n consecutive
+ *            values of a row (blocks from k = 0) by the Walsh-Hadamard
+ *            matrix of order n, Sylvester order H[i][j] = (-1)^popcount(i&j),
+ *            ahead of the quantizer (the DYNAMIC amax is that of the rotated
+ *            tensor).  Computed in binary32 by the fast transform (for
+ *            h = 1, 2, 4, ... < n every pair (i, i + h) with bit h of i clear
+ *            becomes (RN(a + b), RN(a - b))), then multiplied by 2^-shift
+ *            (exact): shift = ceil(log2(n) / 2) for activations
+ *            (fp4_quantize_act_ex, fp4_gemm_fused_ex) and floor(log2(n) / 2)
+ *            for weights (fp4_quantize_weights_ex), so that a rotated
+ *            activation times a weight rotated with the same n gives the
+ *            plain product: H H^T = n I.  Needs K % n == 0 (always true for
+ *            K % 32 == 0).  "FP4 on a consumer RTX 5090: the Blackwell
+ *            headline loses to plain int4", section "Finding 3 -- the
+ *            real-FP4 path (QuTLASS MXFP4)" (the online Hadamard rotation +
+ *            activation quantization every layer pays).
+ *  mx_rule   MXFP4 shared-exponent rule.  FP4_MX_RULE_OCP: e = floor(log2
+ *            amax_b) - 2 (values in (6, 8) * 2^e clip to 6).
+ *            FP4_MX_RULE_OAS (overflow-aware): the smallest e with
+ *            amax_b <= 6 * 2^e, so no value of the block saturates ("FP4
+ *            n'existe pas", section "L'ecart de qualite -- et comment il se
+ *            reduit").  Both clamp e to [-127, 127].  Must be
+ *            FP4_MX_RULE_OCP for NVFP4 (FP4_ERR_INVALID_ARG otherwise). */
+typedef enum { FP4_MX_RULE_OCP = 0, FP4_MX_RULE_OAS = 1 } fp4_mx_rule_t;
+typedef struct {
+    int hadamard;
+    fp4_mx_rule_t mx_rule;
+} fp4_quant_opts_t;
+
+/* fp4_quantize_act with options (above).  opts == NULL is fp4_quantize_act.
+ * FP4_ERR_INVALID_ARG for a hadamard other than 0, 16, 32 or an unknown
+ * rule. */
+fp4_status_t fp4_quantize_act_ex(const void* x, int rows, int K, fp4_format_t fmt,
+                                 fp4_scale_layout_t layout, fp4_global_mode_t gmode,
+                                 const fp4_quant_opts_t* opts, float* g, uint8_t* codes,
+                                 uint8_t* scales, void* ws, size_t ws_bytes, void* stream);
+
 /* One-time weight quantization at load time ("fp4-cuda-kernel" forum post:
  * quantize weights once at model load).  Same arithmetic as
  * fp4_quantize_act with DYNAMIC global scale and scales written in the MMA
@@ -116,6 +155,12 @@ fp4_status_t fp4_quantize_act(const void* x, int rows, int K, fp4_format_t fmt,
 fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt,
                                   uint8_t* codes, uint8_t* scales, float* g,
                                   void* ws, size_t ws_bytes, void* stream);
+
+/* fp4_quantize_weights with options (the weight shift of the rotation). */
+fp4_status_t fp4_quantize_weights_ex(const void* w, int N, int K, fp4_format_t fmt,
+                                     const fp4_quant_opts_t* opts, uint8_t* codes,
+                                     uint8_t* scales, float* g, void* ws, size_t ws_bytes,
+                                     void* stream);
 
 /* Block-scaled FP4 GEMM on the tcgen05 tensor cores:
  *     C[M, N] = alpha * A_hat[M, K] . W_hat[N, K]^T
@@ -168,6 +213,78 @@ fp4_status_t fp4_gemm_fused(const void* a, const uint8_t* w_codes, const uint8_t
                             fp4_global_mode_t gmode, float* g_a,
                             void* C, int ldc, fp4_out_t out,
                             void* ws, size_t ws_bytes, int max_sms, void* stream);
+
+/* fp4_gemm_fused with quantizer options for the activation (the activation
+ * shift of the rotation; the weights must have been quantized by
+ * fp4_quantize_weights_ex with the same hadamard order).  opts == NULL is
+ * fp4_gemm_fused. */
+fp4_status_t fp4_gemm_fused_ex(const void* a, const uint8_t* w_codes, const uint8_t* w_scales,
+                               const float* g_w, int M, int N, int K, fp4_format_t fmt,
+                               fp4_global_mode_t gmode, const fp4_quant_opts_t* opts,
+                               float* g_a, void* C, int ldc, fp4_out_t out,
+                               void* ws, size_t ws_bytes, int max_sms, void* stream);
+
+/* Block-scaled FP4 GEMM whose epilogue emits the next layer's FP4
+ * activation: C = alpha * A_hat . W_hat^T as fp4_gemm computes it, rounded
+ * to bf16 exactly as fp4_gemm writes it, then quantized in the same launch
+ * (no HBM round trip of C) with the activation quantizer's arithmetic:
+ * NVFP4 with the STATIC global scale *g_out (a DYNAMIC scale would need the
+ * whole C before any block could be coded), or MXFP4 (g_out ignored, may be
+ * NULL), with out_opts' rotation (activation shift) and MXFP4 rule.  The
+ * results equal fp4_quantize_act_ex(STATIC g_out) applied to that bf16 C,
+ * bit for bit.
+ *   out_codes   [M, N/2] packed codes; out_scales in out_layout for a
+ *               [M, N] tensor (the MMA order pads rows to 128 and scale
+ *               columns to 4, written as 0), i.e. what the next fp4_gemm
+ *               takes as its activation with K = N.
+ *   C, ldc      optional: when C is not NULL the bf16 C is stored as well
+ *               (row-major, leading dimension ldc).
+ * N % 32 == 0 (N is the next layer's K).  The launch shape is fp4_gemm's
+ * without a K split (every output row of a tile is quantized by the thread
+ * that holds it), so for shapes where fp4_gemm_plan reports a split the
+ * FP32 summation order can differ from fp4_gemm's.  ws unused (may be
+ * NULL).  "FP4 n'existe pas : il existe des FP4, et chaque runtime choisit
+ * son dialecte", section "TensorRT-LLM 1.3 : NVFP4 natif, verrouille
+ * NVIDIA" (quantization, scaling, matmul and de-scaling in one launch, no
+ * HBM round trip between the steps). */
+fp4_status_t fp4_gemm_quant(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                            const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
+                            int M, int N, int K, fp4_format_t fmt, fp4_format_t out_fmt,
+                            fp4_scale_layout_t out_layout, const fp4_quant_opts_t* out_opts,
+                            const float* g_out, uint8_t* out_codes, uint8_t* out_scales,
+                            void* C, int ldc, void* ws, size_t ws_bytes, int max_sms,
+                            void* stream);
+
+/* Grouped block-scaled FP4 GEMM (mixture of experts: many per-expert GEMMs
+ * in one launch).  Group e (0 <= e < E) is rows [offsets[e], offsets[e+1])
+ * of A and C and expert weight e:
+ *     C[r, :] = alpha_e * A_hat[r, :] . W_hat_e^T   for r in group e,
+ * alpha_e = RN(g_a * g_w[e]) (NVFP4; 1 for MXFP4), FP32 accumulation in
+ * tensor memory, bf16 (round to nearest even) or fp32 out.
+ *   a_codes, a_scales, g_a   the routed activation [M, K] as written by
+ *               fp4_quantize_act (MMA scale order, one global scale for all
+ *               rows); groups may start on any row.
+ *   w_codes     E experts' packed codes back to back, [E, N, K/2];
+ *   w_scales    E per-expert MMA-order scale blocks back to back, each
+ *               fp4_scale_bytes(N, K, fmt, FP4_SCALES_MMA) bytes (what
+ *               fp4_quantize_weights writes for one expert);
+ *   g_w         E global scales (NVFP4; may be NULL for MXFP4);
+ *   offsets     DEVICE array of E + 1 ints, offsets[0] = 0, non-decreasing,
+ *               offsets[E] = M (routing results stay on the device; no host
+ *               synchronization).  Out-of-range or decreasing entries are
+ *               clamped into [0, M] and made non-decreasing, so no row
+ *               outside A and C is read or written.
+ * 1 <= E <= 256, N % 8 == 0, K % 32 == 0.  Empty groups are allowed.  The
+ * tiles are 128 x 128 with all of K (no split), so each element's FP32 sum
+ * runs in the same order as fp4_gemm's 128-row kernel.  ws unused (may be
+ * NULL).  "FP4 n'existe pas : il existe des FP4, et chaque runtime choisit
+ * son dialecte", section "Les runtimes et leurs dialectes : qui parle quoi"
+ * (fused NVFP4 MoE kernels, W4A4 MegaMoE). */
+fp4_status_t fp4_gemm_grouped(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                              const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
+                              const int* offsets, int E, int M, int N, int K, fp4_format_t fmt,
+                              void* C, int ldc, fp4_out_t out, void* ws, size_t ws_bytes,
+                              int max_sms, void* stream);
 
 /* The launch shape fp4_gemm takes for an M x N x K problem on the current
  * device, for tests and profiling (nothing is launched; the pages have no

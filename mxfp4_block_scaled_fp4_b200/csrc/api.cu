@@ -84,6 +84,73 @@ size_t quant_ws_bytes() { return fp4::quant_workspace_bytes(); }
 
 fp4_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA; }
 
+// Quantizer options -> (rotation order, 2^-shift, rule); weights take the
+// smaller shift of the rotation, activations the larger (they add up to
+// log2(n)).
+struct Opts {
+  int rot = 0;
+  float rot_scale = 1.0f;
+  int rule = 0;
+};
+fp4_status_t parse_opts(const fp4_quant_opts_t* o, fp4_format_t fmt, bool weights, Opts* out) {
+  *out = Opts{};
+  if (!o) return FP4_OK;
+  if (o->hadamard != 0 && o->hadamard != 16 && o->hadamard != 32) return FP4_ERR_INVALID_ARG;
+  if (o->mx_rule != FP4_MX_RULE_OCP && o->mx_rule != FP4_MX_RULE_OAS) return FP4_ERR_INVALID_ARG;
+  if (fmt == FP4_NVFP4 && o->mx_rule != FP4_MX_RULE_OCP) return FP4_ERR_INVALID_ARG;
+  out->rot = o->hadamard;
+  out->rule = o->mx_rule == FP4_MX_RULE_OAS ? 1 : 0;
+  if (o->hadamard) {
+    const int lg = o->hadamard == 16 ? 4 : 5;
+    const int shift = weights ? lg / 2 : (lg + 1) / 2;
+    out->rot_scale = 1.0f / static_cast<float>(1 << shift);
+  }
+  return FP4_OK;
+}
+
+fp4_status_t quantize_common(const void* x, int rows, int K, fp4_format_t fmt,
+                             fp4_scale_layout_t layout, fp4_global_mode_t gmode,
+                             const fp4_quant_opts_t* opts, bool weights, float* g,
+                             uint8_t* codes, uint8_t* scales, void* ws, size_t ws_bytes,
+                             void* stream) {
+  fp4_status_t st;
+  if ((st = check_format(fmt)) != FP4_OK) return st;
+  if (layout != FP4_SCALES_MMA && layout != FP4_SCALES_ROWMAJOR) return FP4_ERR_INVALID_ARG;
+  if (gmode != FP4_GLOBAL_DYNAMIC && gmode != FP4_GLOBAL_STATIC) return FP4_ERR_INVALID_ARG;
+  Opts op;
+  if ((st = parse_opts(opts, fmt, weights, &op)) != FP4_OK) return st;
+  if ((st = check_rows_k(rows, K)) != FP4_OK) return st;
+  if (rows == 0) return FP4_OK;   // nothing is read or written
+  const bool nv = fmt == FP4_NVFP4;
+  const bool dyn = nv && gmode == FP4_GLOBAL_DYNAMIC;
+  if (!x || !codes || !scales || (nv && !g) || (dyn && !ws)) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (nv && !aligned4(g)) ||
+      (dyn && !aligned16(ws)))
+    return FP4_ERR_MISALIGNED;
+  if (dyn && ws_bytes < quant_ws_bytes()) return FP4_ERR_WORKSPACE_TOO_SMALL;
+  if ((st = device_ok()) != FP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fp4::QuantArgs a{};
+  a.x = x;
+  a.rows = rows;
+  a.K = K;
+  a.fmt = fmt;
+  a.layout = layout;
+  a.dynamic = dyn ? 1 : 0;
+  a.g = g;
+  a.codes = codes;
+  a.scales = scales;
+  a.rot = op.rot;
+  a.rot_scale = op.rot_scale;
+  a.rule = op.rule;
+  // The amax pass (DYNAMIC) and the quantize pass, each a programmatic
+  // dependent of the kernel before it (each waits for its predecessor before
+  // reading), so its launch overlaps the predecessor's tail.  No pass
+  // releases its own dependent early: a fused GEMM may read weights before
+  // its wait.
+  return from_cuda(fp4::launch_quantize_act(a, static_cast<unsigned*>(ws), s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -114,44 +181,31 @@ fp4_status_t fp4_quantize_act(const void* x, int rows, int K, fp4_format_t fmt,
                               fp4_scale_layout_t layout, fp4_global_mode_t gmode, float* g,
                               uint8_t* codes, uint8_t* scales, void* ws, size_t ws_bytes,
                               void* stream) {
-  fp4_status_t st;
-  if ((st = check_format(fmt)) != FP4_OK) return st;
-  if (layout != FP4_SCALES_MMA && layout != FP4_SCALES_ROWMAJOR) return FP4_ERR_INVALID_ARG;
-  if (gmode != FP4_GLOBAL_DYNAMIC && gmode != FP4_GLOBAL_STATIC) return FP4_ERR_INVALID_ARG;
-  if ((st = check_rows_k(rows, K)) != FP4_OK) return st;
-  if (rows == 0) return FP4_OK;   // nothing is read or written
-  const bool nv = fmt == FP4_NVFP4;
-  const bool dyn = nv && gmode == FP4_GLOBAL_DYNAMIC;
-  if (!x || !codes || !scales || (nv && !g) || (dyn && !ws)) return FP4_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (nv && !aligned4(g)) ||
-      (dyn && !aligned16(ws)))
-    return FP4_ERR_MISALIGNED;
-  if (dyn && ws_bytes < quant_ws_bytes()) return FP4_ERR_WORKSPACE_TOO_SMALL;
-  if ((st = device_ok()) != FP4_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  fp4::QuantArgs a{};
-  a.x = x;
-  a.rows = rows;
-  a.K = K;
-  a.fmt = fmt;
-  a.layout = layout;
-  a.dynamic = dyn ? 1 : 0;
-  a.g = g;
-  a.codes = codes;
-  a.scales = scales;
-  // The amax pass (DYNAMIC) and the quantize pass, each a programmatic
-  // dependent of the kernel before it (each waits for its predecessor before
-  // reading), so its launch overlaps the predecessor's tail.  No pass
-  // releases its own dependent early: a fused GEMM may read weights before
-  // its wait.
-  return from_cuda(fp4::launch_quantize_act(a, static_cast<unsigned*>(ws), s));
+  return quantize_common(x, rows, K, fmt, layout, gmode, nullptr, false, g, codes, scales, ws,
+                         ws_bytes, stream);
+}
+
+fp4_status_t fp4_quantize_act_ex(const void* x, int rows, int K, fp4_format_t fmt,
+                                 fp4_scale_layout_t layout, fp4_global_mode_t gmode,
+                                 const fp4_quant_opts_t* opts, float* g, uint8_t* codes,
+                                 uint8_t* scales, void* ws, size_t ws_bytes, void* stream) {
+  return quantize_common(x, rows, K, fmt, layout, gmode, opts, false, g, codes, scales, ws,
+                         ws_bytes, stream);
 }
 
 fp4_status_t fp4_quantize_weights(const void* w, int N, int K, fp4_format_t fmt, uint8_t* codes,
                                   uint8_t* scales, float* g, void* ws, size_t ws_bytes,
                                   void* stream) {
-  return fp4_quantize_act(w, N, K, fmt, FP4_SCALES_MMA, FP4_GLOBAL_DYNAMIC, g, codes, scales, ws,
-                          ws_bytes, stream);
+  return quantize_common(w, N, K, fmt, FP4_SCALES_MMA, FP4_GLOBAL_DYNAMIC, nullptr, true, g,
+                         codes, scales, ws, ws_bytes, stream);
+}
+
+fp4_status_t fp4_quantize_weights_ex(const void* w, int N, int K, fp4_format_t fmt,
+                                     const fp4_quant_opts_t* opts, uint8_t* codes,
+                                     uint8_t* scales, float* g, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  return quantize_common(w, N, K, fmt, FP4_SCALES_MMA, FP4_GLOBAL_DYNAMIC, opts, true, g, codes,
+                         scales, ws, ws_bytes, stream);
 }
 
 fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
@@ -190,9 +244,111 @@ fp4_status_t fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const flo
   a.fmt = fmt;
   a.C = C;
   a.ldc = ldc;
-  a.out_f32 = out == FP4_OUT_F32;
+  a.out_mode = out == FP4_OUT_F32 ? 1 : 0;
   a.max_sms = max_sms;
   return from_cuda(fp4::launch_gemm(a, static_cast<cudaStream_t>(stream)));
+}
+
+fp4_status_t fp4_gemm_quant(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                            const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
+                            int M, int N, int K, fp4_format_t fmt, fp4_format_t out_fmt,
+                            fp4_scale_layout_t out_layout, const fp4_quant_opts_t* out_opts,
+                            const float* g_out, uint8_t* out_codes, uint8_t* out_scales, void* C,
+                            int ldc, void* ws, size_t ws_bytes, int max_sms, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  fp4_status_t st;
+  if ((st = check_format(fmt)) != FP4_OK || (st = check_format(out_fmt)) != FP4_OK) return st;
+  if (out_layout != FP4_SCALES_MMA && out_layout != FP4_SCALES_ROWMAJOR) return FP4_ERR_INVALID_ARG;
+  Opts op;
+  if ((st = parse_opts(out_opts, out_fmt, false, &op)) != FP4_OK) return st;
+  if (max_sms < 0) return FP4_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (N % 32 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;   // N is the next layer's K
+  if (M == 0 || N == 0) return FP4_OK;
+  const bool nv = fmt == FP4_NVFP4, nv_out = out_fmt == FP4_NVFP4;
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !out_codes || !out_scales ||
+      (nv && (!g_a || !g_w)) || (nv_out && !g_out))
+    return FP4_ERR_INVALID_ARG;
+  if (C && ldc < N) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(out_codes) || !aligned16(out_scales) ||
+      (C && (!aligned16(C) || (static_cast<long long>(ldc) * 2) % 16 != 0)) ||
+      (nv && (!aligned4(g_a) || !aligned4(g_w))) || (nv_out && !aligned4(g_out)))
+    return FP4_ERR_MISALIGNED;
+  if ((st = device_ok()) != FP4_OK) return st;
+  fp4::GemmArgs a{};
+  a.a_codes = a_codes;
+  a.a_scales = a_scales;
+  a.g_a = g_a;
+  a.w_codes = w_codes;
+  a.w_scales = w_scales;
+  a.g_w = g_w;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.fmt = fmt;
+  a.C = C;
+  a.ldc = C ? ldc : N;
+  a.out_mode = nv_out ? 2 : 3;
+  a.max_sms = max_sms;
+  a.qo.codes = out_codes;
+  a.qo.scales = out_scales;
+  a.qo.g = g_out;
+  a.qo.fmt = nv_out ? 0 : 1;
+  a.qo.layout = out_layout == FP4_SCALES_ROWMAJOR ? 1 : 0;
+  a.qo.rule = op.rule;
+  a.qo.rot = op.rot;
+  a.qo.rot_scale = op.rot_scale;
+  a.qo.nsf = fp4::nsf_of(N, a.qo.fmt);
+  a.qo.ncb = fp4::ncb_of(a.qo.nsf);
+  return from_cuda(fp4::launch_gemm(a, static_cast<cudaStream_t>(stream)));
+}
+
+fp4_status_t fp4_gemm_grouped(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                              const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
+                              const int* offsets, int E, int M, int N, int K, fp4_format_t fmt,
+                              void* C, int ldc, fp4_out_t out, void* ws, size_t ws_bytes,
+                              int max_sms, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  fp4_status_t st;
+  if ((st = check_format(fmt)) != FP4_OK) return st;
+  if (out != FP4_OUT_BF16 && out != FP4_OUT_F32) return FP4_ERR_INVALID_ARG;
+  if (max_sms < 0) return FP4_ERR_INVALID_ARG;
+  if (E < 1 || E > fp4::kGroupedMaxGroups) return FP4_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return FP4_OK;   // nothing is read or written
+  const bool nv = fmt == FP4_NVFP4;
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !offsets || !C ||
+      (nv && (!g_a || !g_w)))
+    return FP4_ERR_INVALID_ARG;
+  if (ldc < N) return FP4_ERR_INVALID_ARG;
+  const int esize = out == FP4_OUT_F32 ? 4 : 2;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(C) || !aligned4(offsets) || (static_cast<long long>(ldc) * esize) % 16 != 0 ||
+      (nv && (!aligned4(g_a) || !aligned4(g_w))))
+    return FP4_ERR_MISALIGNED;
+  if ((st = device_ok()) != FP4_OK) return st;
+  fp4::GroupedArgs a{};
+  a.a_codes = a_codes;
+  a.a_scales = a_scales;
+  a.g_a = g_a;
+  a.w_codes = w_codes;
+  a.w_scales = w_scales;
+  a.g_w = g_w;
+  a.offsets = offsets;
+  a.E = E;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.fmt = fmt;
+  a.C = C;
+  a.ldc = ldc;
+  a.out_f32 = out == FP4_OUT_F32;
+  a.max_sms = max_sms;
+  return from_cuda(fp4::launch_gemm_grouped(a, static_cast<cudaStream_t>(stream)));
 }
 
 fp4_status_t fp4_gemm_plan(int M, int N, int K, fp4_format_t fmt, int max_sms, int* tile_m,
@@ -210,8 +366,19 @@ fp4_status_t fp4_gemm_fused(const void* x, const uint8_t* w_codes, const uint8_t
                             const float* g_w, int M, int N, int K, fp4_format_t fmt,
                             fp4_global_mode_t gmode, float* g_a, void* C, int ldc, fp4_out_t out,
                             void* ws, size_t ws_bytes, int max_sms, void* stream) {
+  return fp4_gemm_fused_ex(x, w_codes, w_scales, g_w, M, N, K, fmt, gmode, nullptr, g_a, C, ldc,
+                           out, ws, ws_bytes, max_sms, stream);
+}
+
+fp4_status_t fp4_gemm_fused_ex(const void* x, const uint8_t* w_codes, const uint8_t* w_scales,
+                               const float* g_w, int M, int N, int K, fp4_format_t fmt,
+                               fp4_global_mode_t gmode, const fp4_quant_opts_t* opts, float* g_a,
+                               void* C, int ldc, fp4_out_t out, void* ws, size_t ws_bytes,
+                               int max_sms, void* stream) {
   fp4_status_t st;
   if ((st = check_format(fmt)) != FP4_OK) return st;
+  Opts op;
+  if ((st = parse_opts(opts, fmt, false, &op)) != FP4_OK) return st;
   if (out != FP4_OUT_BF16 && out != FP4_OUT_F32) return FP4_ERR_INVALID_ARG;
   if (gmode != FP4_GLOBAL_DYNAMIC && gmode != FP4_GLOBAL_STATIC) return FP4_ERR_INVALID_ARG;
   if (max_sms < 0) return FP4_ERR_INVALID_ARG;
@@ -247,6 +414,9 @@ fp4_status_t fp4_gemm_fused(const void* x, const uint8_t* w_codes, const uint8_t
   a.ws = ws;
   a.ws_bytes = ws_bytes;
   a.max_sms = max_sms;
+  a.rot = op.rot;
+  a.rot_scale = op.rot_scale;
+  a.rule = op.rule;
   return from_cuda(fp4::launch_gemm_fused(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -113,10 +113,122 @@ __device__ __forceinline__ float nvfp4_recip(unsigned s, float g) {
   return (sv == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sv, g));
 }
 
-// One 32-value MXFP4 block: E8M0 scale byte and r = 2^-e.
-__device__ __forceinline__ unsigned mxfp4_scale(unsigned amax_bits, float* r) {
-  const float b = __uint_as_float(amax_bits << 16);
-  int e = (b == 0.0f) ? -127 : floor_log2(b) - 2;
+
+// ------------------------------------------------------------------------
+// Online rotation (the Hadamard rotation ahead of the activation quantizer of
+// "FP4 on a consumer RTX 5090: the Blackwell headline loses to plain int4",
+// section "Finding 3 -- the real-FP4 path (QuTLASS MXFP4)").  Block-diagonal
+// Walsh-Hadamard of order n in {16, 32} along K, Sylvester order, computed in
+// binary32 as the fast transform: for h = 1, 2, 4, ... < n every pair
+// (i, i + h) with bit h of i clear becomes (RN(a + b), RN(a - b)); then a
+// multiply by 2^-shift (exact).  A thread holds one 16-value unit; with
+// n = 32 the last stage pairs the unit with its lane neighbour (lane ^ 1),
+// whose unit is the other half of the same 32-value block.
+
+// 16 bf16 (8 words, element 2i in the low half of word i) -> 16 floats.
+__device__ __forceinline__ void unpack16(uint4 p, uint4 q, float f[16]) {
+  const unsigned w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// The in-unit stages h = 1, 2, 4, 8 of the transform, then (n = 16) the
+// scaling; n = 32 adds the cross-lane stage h = 16 (every lane of the warp
+// must take part) before it.  `odd` = this unit is the upper half of its
+// 32-value block.
+template <int N>
+__device__ __forceinline__ void rotate_unit(float f[16], float scale, bool odd) {
+#pragma unroll
+  for (int h = 1; h < 16; h *= 2) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if ((i & h) == 0) {
+        const float a = f[i], b = f[i + h];
+        f[i] = __fadd_rn(a, b);
+        f[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+  if (N == 32) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float o = __shfl_xor_sync(0xFFFFFFFFu, f[i], 1);
+      // lower half: own + other; upper half: lower (the other) - own
+      f[i] = odd ? __fsub_rn(o, f[i]) : __fadd_rn(f[i], o);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(f[i], scale);   // exact: a power of two
+}
+
+// Largest magnitude of 16 floats as binary32 magnitude bits (Inf and NaN
+// order above every finite value).
+__device__ __forceinline__ unsigned mag_max16(const float f[16]) {
+  unsigned m = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m = max(m, __float_as_uint(f[i]) & 0x7FFFFFFFu);
+  return m;
+}
+
+// 8 floats times r -> 8 packed E2M1 codes (element i in nibble i); the
+// rounding and sign rules of quant8.
+__device__ __forceinline__ unsigned quant8_f32(const float* f, float r) {
+  unsigned out;
+  asm("{\n\t"
+      ".reg .b64 x0, x1, x2, x3, rr;\n\t"
+      ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+      ".reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b64 rr, {%9, %9};\n\t"
+      "mov.b64 x0, {%1, %2};\n\t mov.b64 x1, {%3, %4};\n\t"
+      "mov.b64 x2, {%5, %6};\n\t mov.b64 x3, {%7, %8};\n\t"
+      "mul.rn.f32x2 x0, x0, rr;\n\t mul.rn.f32x2 x1, x1, rr;\n\t"
+      "mul.rn.f32x2 x2, x2, rr;\n\t mul.rn.f32x2 x3, x3, rr;\n\t"
+      "mov.b64 {l0, h0}, x0;\n\t mov.b64 {l1, h1}, x1;\n\t"
+      "mov.b64 {l2, h2}, x2;\n\t mov.b64 {l3, h3}, x3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, h0, l0;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, h1, l1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, h2, l2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, h3, l3;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(f[0]), "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7]),
+        "f"(r));
+  return out;
+}
+
+// One 16-value NVFP4 block of binary32 values: s = E4M3(RN(b / RN(6 g)))
+// with b the block's largest magnitude (binary32 bits).
+__device__ __forceinline__ unsigned nvfp4_scale_byte_f32(unsigned b_bits, float six_g, float y6,
+                                                         bool fast_b) {
+  return to_e4m3(div_rn(__uint_as_float(b_bits), six_g, y6, fast_b));
+}
+
+// One 32-value MXFP4 block of binary32 values with block maximum b (bits):
+// rule 0 = OCP, e = floor(log2 b) - 2; rule 1 = overflow-aware (OAS), the
+// smallest e with b <= 6 * 2^e, i.e. one more than OCP's when the
+// significand of b exceeds 1.5 ("FP4 n'existe pas", section "L'ecart de
+// qualite -- et comment il se reduit").  Clamped to [-127, 127]; E8M0 byte
+// e + 127, r = 2^-e.
+__device__ __forceinline__ unsigned mxfp4_scale_f32(unsigned b_bits, int rule, float* r) {
+  const float b = __uint_as_float(b_bits);
+  int e = -127;
+  if (b != 0.0f) {
+    e = floor_log2(b) - 2;
+    if (rule) {
+      const unsigned ex = (b_bits >> 23) & 0xFFu, man = b_bits & 0x7FFFFFu;
+      bool above;   // significand of b > 1.5
+      if (ex != 0) {
+        above = man > 0x400000u;
+      } else {
+        const int msb = 31 - __clz(man);
+        above = msb >= 1 && (man & ((1u << msb) - 1u)) > (1u << (msb - 1));
+      }
+      e += above ? 1 : 0;
+    }
+  }
   e = max(-127, min(127, e));
   *r = __uint_as_float(static_cast<unsigned>(127 - e) << 23);
   return static_cast<unsigned>(e + 127);

@@ -102,6 +102,8 @@ struct DParams {
   int dynamic, out_f32;
   int n_tiles, k_steps, splits, nmma_n, ncb;
   unsigned* watchdog;
+  float rot_scale;           // rotation (ROT = 16 or 32): 2^-shift
+  int rule;                  // MXFP4 scale rule: 0 OCP, 1 overflow-aware
 };
 
 __device__ __forceinline__ void workers_sync() {   // named barrier of the 4 worker warps
@@ -130,7 +132,7 @@ __device__ __forceinline__ void store_out(const DParams& p, int m, int n, float 
     static_cast<__nv_bfloat16*>(p.C)[m * p.ldc + n] = __float2bfloat16_rn(c);
 }
 
-template <int FMT>
+template <int FMT, int ROT>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_w, const DParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -301,25 +303,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (FMT == 0) {
       if (p.dynamic) {
         unsigned m = 0;
-        const long long n_vec = static_cast<long long>(p.M) * p.K / 8;
-        // eight 16-byte loads in flight per thread
-        for (long long v = wt; v < n_vec; v += 1024) {
-          uint4 t[8];
+        if (ROT == 0) {
+          const long long n_vec = static_cast<long long>(p.M) * p.K / 8;
+          // eight 16-byte loads in flight per thread
+          for (long long v = wt; v < n_vec; v += 1024) {
+            uint4 t[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            t[j] = (v + 128 * j < n_vec) ? ld_x16(p.x + (v + 128 * j) * 8) : make_uint4(0u, 0u, 0u, 0u);
+            for (int j = 0; j < 8; ++j)
+              t[j] = (v + 128 * j < n_vec) ? ld_x16(p.x + (v + 128 * j) * 8) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) m = max_u16x2(m, mag_max8(t[j]));
+            for (int j = 0; j < 8; ++j) m = max_u16x2(m, mag_max8(t[j]));
+          }
+          m = fold_u16x2(m);
+        } else {
+          // rotated values: 16-value units, four (eight loads) in flight per
+          // thread; whole warps iterate together (a 32-rotation pairs lanes)
+          const long long n_units = static_cast<long long>(p.M) * p.K / 16;
+          for (long long base = 0; base < n_units; base += 512) {
+            uint4 t[4][2];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const long long u = base + wt + 128 * j;
+              const bool in = u < n_units;
+              t[j][0] = in ? ld_x16(p.x + u * 16) : make_uint4(0u, 0u, 0u, 0u);
+              t[j][1] = in ? ld_x16(p.x + u * 16 + 8) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float f[16];
+              unpack16(t[j][0], t[j][1], f);
+              rotate_unit<ROT>(f, p.rot_scale, (lane & 1) != 0);
+              m = max(m, mag_max16(f));
+            }
+          }
         }
-        m = fold_u16x2(m);
         for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
         if (lane == 0) red[warp - 2] = m;
         workers_sync();
         m = max(max(red[0], red[1]), max(red[2], red[3]));
         // CTA 0 reports a non-finite input; every CTA clamps alike
-        if (m > kBf16MaxFinite)
-          m = (blockIdx.x == 0 && wt == 0) ? amax_checked(m, p.watchdog) : kBf16MaxFinite;
-        const float amax = __uint_as_float(m << 16);
+        float amax;
+        if (ROT == 0) {
+          if (m > kBf16MaxFinite)
+            m = (blockIdx.x == 0 && wt == 0) ? amax_checked(m, p.watchdog) : kBf16MaxFinite;
+          amax = __uint_as_float(m << 16);
+        } else {
+          if (m > kF32MaxFinite)
+            m = (blockIdx.x == 0 && wt == 0) ? amax_checked_f32(m, p.watchdog) : kF32MaxFinite;
+          amax = __uint_as_float(m);
+        }
         g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
         if (blockIdx.x == 0 && wt == 0) *p.g_a = g;
       } else {
@@ -351,24 +383,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           nx0 = ld_x16(src);
           nx1 = ld_x16(src + 8);
         }
-        unsigned mx = fold_u16x2(max_u16x2(mag_max8(a0), mag_max8(a1)));
         unsigned sbyte;
         float r;
         uint2 packed;
-        if (FMT == 0) {
-          sbyte = 0u;
-          packed = make_uint2(0u, 0u);
-          if (valid) {
-            sbyte = nvfp4_scale_byte(mx, six_g, y6, fast_b);
-            r = r_tab[sbyte & 127u];
-            if (r != 0.0f)
-              packed = make_uint2(quant8(a0.x, a0.y, a0.z, a0.w, r), quant8(a1.x, a1.y, a1.z, a1.w, r));
+        if (ROT == 0) {
+          unsigned mx = fold_u16x2(max_u16x2(mag_max8(a0), mag_max8(a1)));
+          if (FMT == 0) {
+            sbyte = 0u;
+            packed = make_uint2(0u, 0u);
+            if (valid) {
+              sbyte = nvfp4_scale_byte(mx, six_g, y6, fast_b);
+              r = r_tab[sbyte & 127u];
+              if (r != 0.0f)
+                packed = make_uint2(quant8(a0.x, a0.y, a0.z, a0.w, r), quant8(a1.x, a1.y, a1.z, a1.w, r));
+            }
+          } else {
+            // a 32-value block is a pair of adjacent units = adjacent lanes
+            mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+            sbyte = mxfp4_scale_f32(mx << 16, p.rule, &r);
+            packed = make_uint2(quant8(a0.x, a0.y, a0.z, a0.w, r), quant8(a1.x, a1.y, a1.z, a1.w, r));
           }
         } else {
-          // a 32-value block is a pair of adjacent units = adjacent lanes
-          mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-          sbyte = mxfp4_scale(mx, &r);
-          packed = make_uint2(quant8(a0.x, a0.y, a0.z, a0.w, r), quant8(a1.x, a1.y, a1.z, a1.w, r));
+          // rotated unit (lanes 2i, 2i+1 hold the halves of a 32-value block;
+          // every lane takes part, invalid ones with zeros)
+          float f[16];
+          unpack16(a0, a1, f);
+          rotate_unit<ROT>(f, p.rot_scale, (lane & 1) != 0);
+          unsigned mx = mag_max16(f);
+          if (FMT == 0) {
+            sbyte = nvfp4_scale_byte_f32(mx, six_g, y6, fast_b);
+            r = r_tab[sbyte & 127u];
+            packed = (r == 0.0f) ? make_uint2(0u, 0u) : make_uint2(quant8_f32(f, r), quant8_f32(f + 8, r));
+          } else {
+            mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+            sbyte = mxfp4_scale_f32(mx, p.rule, &r);
+            packed = make_uint2(quant8_f32(f, r), quant8_f32(f + 8, r));
+          }
         }
         if (valid) {
           const int step = i >> 4, iu = i & 15;
@@ -523,9 +573,15 @@ cudaError_t launch_decode(const FusedArgs& f, cudaStream_t s) {
   p.ncb = ncb_of(nsf_of(f.K, f.fmt));
   p.watchdog = watchdog_ptr();
   if (!p.watchdog) return cudaErrorInvalidSymbol;
+  p.rot_scale = f.rot_scale;
+  p.rule = f.rule;
   CUtensorMap mw;
   if (!make_code_map(&mw, f.w_codes, f.N, f.K, DBM)) return cudaErrorInvalidValue;
-  auto kern = (f.fmt == 0) ? decode_kernel<0> : decode_kernel<1>;
+  using Kern = void (*)(const CUtensorMap, const DParams);
+  static const Kern table[3][2] = {{decode_kernel<0, 0>, decode_kernel<1, 0>},
+                                   {decode_kernel<0, 16>, decode_kernel<1, 16>},
+                                   {decode_kernel<0, 32>, decode_kernel<1, 32>}};
+  const Kern kern = table[f.rot == 32 ? 2 : (f.rot == 16 ? 1 : 0)][f.fmt != 0];
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};

@@ -457,6 +457,9 @@ cudaError_t launch_gemm_fused(const FusedArgs& f, cudaStream_t s) {
   q.g = f.g_a;
   q.codes = x_codes;
   q.scales = x_scales;
+  q.rot = f.rot;
+  q.rot_scale = f.rot_scale;
+  q.rule = f.rule;
   // scale columns past K of real rows are still zeroed (they meet zero codes,
   // and 0 x NaN would not be 0); rows >= M only reach output columns that
   // are never stored

@@ -59,6 +59,7 @@ constexpr uint32_t ACC_COL = 0;         // up to 256 fp32 columns
 constexpr uint32_t SF_COL = 256;        // per stage: 16 columns A scales + 16 or 32 B scales
 constexpr int kGemmThreads = 352;       // 11 warps: TMA, MMA, 4 epilogue, 4 scale staging, scale TMA
 constexpr int GROUP_M = 16;             // tile raster: 16 M-tiles share their W tiles in L2
+constexpr int kMaxGroups = kGroupedMaxGroups;   // experts of a grouped launch
 
 // Output tiles are 128 x BN.  BN = 256 is the throughput shape; 128 and 64
 // give problems with few 256-wide tiles more CTAs (and smaller split-K
@@ -66,15 +67,20 @@ constexpr int GROUP_M = 16;             // tile raster: 16 M-tiles share their W
 // block (two for BN = 256); for BN = 64 the tile is one half of it.  The
 // ring is as deep as shared memory allows, so that narrow tiles keep as
 // many bytes in flight as wide ones.
-template <int BN>
+// G = 1: the grouped (mixture-of-experts) form, whose A tiles start at any
+// row, so a stage holds the A scale atoms of two 128-row blocks, and the
+// group table follows the barriers.
+template <int BN, int G = 0>
 struct Tile {
   static constexpr int B_STAGE = BN * BK_BYTES;
   static constexpr int SF_BLOCKS = (BN == 256) ? 2 : 1;
   static constexpr int SFB_STAGE = SF_BLOCKS * 4 * 512;
-  static constexpr int STAGE_BYTES = A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE;
-  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128) ? 6 : 7;
+  static constexpr int SFA_BYTES = (G ? 2 : 1) * SFA_STAGE;
+  static constexpr int STAGE_BYTES = A_STAGE + B_STAGE + SFA_BYTES + SFB_STAGE;
+  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128) ? (G ? 5 : 6) : 7;
   static constexpr int RING = STAGES * STAGE_BYTES;
-  static constexpr int SMEM = RING + 1024 + 512;   // ring + alignment + barriers
+  static constexpr int GTAB = G ? 4 * (2 * kMaxGroups + 2) : 0;   // group table (ints)
+  static constexpr int SMEM = RING + 1024 + 512 + GTAB;   // ring + alignment + barriers
   // tensor-memory columns between the B scales of consecutive atoms, and
   // per stage (A scales in the first 16)
   static constexpr int SFB_ATOM_COLS = 4 * SF_BLOCKS;
@@ -100,6 +106,14 @@ struct Params {
   int splits;             // CTAs per output tile along K (a cluster), 1 = no split
   int k_per;              // K steps per split
   unsigned* watchdog;
+  // grouped form (G = 1): E groups; group e is rows [offsets[e], offsets[e+1])
+  // of A and C and weights rows [e N, e N + N) of the stacked W, whose
+  // scales start at byte e * w_sf_bytes; g_w holds one global scale per group
+  const int* offsets;
+  int E;
+  long long w_sf_bytes;
+  int a_rowblocks;        // ceil(M / 128)
+  QuantOut qo;            // OUT >= 2: the emitted FP4 activation (C optional)
 };
 
 // Split-K: CTA d of a tile's cluster reduces accumulator rows
@@ -115,6 +129,33 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int
   const int within = t - group * per_group;
   mt = first_m + within % gsize;
   nt = within / gsize;
+}
+
+// A tile of the grouped form: rows [a_row0, a_row_end) of A / C, weight rows
+// from w_row0 of the stacked W, group e.
+struct GTile {
+  int e, a_row0, a_row_end, nt;
+};
+// Tiles of group e occupy [tiles_before[e] * n_tiles, tiles_before[e+1] *
+// n_tiles); within a group the M tiles are the fastest index, so that
+// consecutive CTAs share a W tile in L2.  gtab: tiles_before[0..E] then the
+// group row starts row0[0..E].
+__device__ __forceinline__ GTile gtile(int t, const Params& p, const int* gtab) {
+  const int* before = gtab;
+  const int* row0 = gtab + kMaxGroups + 1;
+  int lo = 0, hi = p.E;                         // largest e with before[e] * n_tiles <= t
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (before[mid] * p.n_tiles <= t) lo = mid; else hi = mid;
+  }
+  GTile g;
+  g.e = lo;
+  const int mt_e = before[lo + 1] - before[lo];
+  const int local = t - before[lo] * p.n_tiles;
+  g.nt = local / mt_e;
+  g.a_row0 = row0[lo] + (local - g.nt * mt_e) * BM;
+  g.a_row_end = row0[lo + 1];
+  return g;
 }
 
 // alpha * 8 accumulator values -> 8 bf16 (one 16-byte store) / 2 float4.
@@ -137,11 +178,15 @@ __device__ __forceinline__ void store8(void* C, long long off, float alpha, cons
   }
 }
 
-template <int FMT, int OUT_F32, int BN>
+// OUT: 0 = bf16 C, 1 = fp32 C, 2 / 3 = C quantized to NVFP4 / MXFP4
+// (out_quant.cuh; no K split), with the bf16 C stored as well when p.C is
+// not null.
+template <int FMT, int OUT, int BN, int G = 0>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                 const Params p) {
-  using T = Tile<BN>;
+  using T = Tile<BN, G>;
+  constexpr int SFA_STAGE = T::SFA_BYTES;
   constexpr int STAGES = T::STAGES;
   constexpr uint32_t SF_STAGE_COLS = T::SF_STAGE_COLS;
   extern __shared__ uint8_t smem_raw[];
@@ -161,10 +206,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* recv = drain + 1;          // split-K: partial sums pushed by the peers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* gtab = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + 512);   // G = 1
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_tiles_total = p.m_tiles * p.n_tiles;
+  int n_tiles_total = p.m_tiles * p.n_tiles;
   // split-K: one tile per cluster, CTA rank = its slice of the K steps;
   // otherwise persistent over the tiles with all K steps
   const bool split = p.splits > 1;
@@ -220,8 +266,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // writes come after the wait.  Without such a launch both are no-ops.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (G) {
+    // the group table from the device-side offsets (clamped to [0, M] and
+    // made non-decreasing, so that malformed offsets cannot address rows
+    // outside A and C): warp 0 scans the groups' M-tile counts 32 at a time
+    if (warp == 0) {
+      int carry = 0, prev_end = 0;
+      for (int base = 0; base < p.E; base += 32) {
+        const int e = base + lane;
+        // lanes past the last group repeat its end, so that lane 31 carries
+        // the true end of the groups into the next chunk and the table
+        const int e0 = min(e, p.E);
+        const int r0 = min(max(p.offsets[e0], 0), p.M);
+        const int r1 = (e < p.E) ? min(max(p.offsets[e + 1], 0), p.M) : r0;
+        // non-decreasing starts: a group starts no earlier than the previous end
+        int start = r0;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xFFFFFFFFu, start, o);
+          if (lane >= o) start = max(start, v);
+        }
+        start = max(start, prev_end);
+        const int end = (e < p.E) ? max(r1, start) : start;
+        int n = (e < p.E) ? (end - start + BM - 1) / BM : 0;
+        int incl = n;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (e < p.E) {
+          gtab[e] = carry + incl - n;
+          gtab[kMaxGroups + 1 + e] = start;
+        }
+        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        prev_end = __shfl_sync(0xFFFFFFFFu, end, 31);
+      }
+      if (lane == 0) {
+        gtab[p.E] = carry;
+        gtab[kMaxGroups + 1 + p.E] = prev_end;
+      }
+    }
+    __syncthreads();
+    n_tiles_total = gtab[p.E] * p.n_tiles;
+  }
   float alpha = 1.0f;
-  if (FMT == 0 && warp >= 2 && warp < 6) alpha = __fmul_rn(*p.g_a, *p.g_w);
+  if (FMT == 0 && warp >= 2 && warp < 6 && !G) alpha = __fmul_rn(*p.g_a, *p.g_w);
+  QuantOutG qg{};
+  if (OUT >= 2 && warp >= 2 && warp < 6) qg = quant_out_g(p.qo);
   bool acc_ok = false;   // split-K epilogue: this CTA's accumulator is complete
 
   constexpr int kAtomsPerStage = (FMT == 0) ? 4 : 2;   // scale atoms per 256 K
@@ -232,14 +322,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;
     for (int t = t_first; t < n_tiles_total; t += t_stride) {
-      int mt, nt;
-      tile_coords(t, p, mt, nt);
+      int mt, nt, a_row0, w_row0;
+      if (G) {
+        const GTile g = gtile(t, p, gtab);
+        nt = g.nt;
+        a_row0 = g.a_row0;
+        w_row0 = g.e * p.N + nt * BN;
+      } else {
+        tile_coords(t, p, mt, nt);
+        a_row0 = mt * BM;
+        w_row0 = nt * BN;
+      }
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.watchdog, WD_PRODUCER)) goto producer_drain;
         {
           mbar_expect_tx(&full[stage], A_STAGE + T::B_STAGE);
-          tma_load_2d(sA + stage * A_STAGE, &tm_a, kb * BK_BYTES, mt * BM, &full[stage]);
-          tma_load_2d(sB + stage * T::B_STAGE, &tm_w, kb * BK_BYTES, nt * BN, &full[stage]);
+          tma_load_2d(sA + stage * A_STAGE, &tm_a, kb * BK_BYTES, a_row0, &full[stage]);
+          tma_load_2d(sB + stage * T::B_STAGE, &tm_w, kb * BK_BYTES, w_row0, &full[stage]);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         }
@@ -267,7 +366,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t armed = 0, armed_parity = 0;
     for (int t = t_first; t < n_tiles_total; t += t_stride) {
       int mt, nt;
-      tile_coords(t, p, mt, nt);
+      int arb, ablocks = 1;             // A scale row block(s) of the tile
+      const uint8_t* wsf = p.w_scales;  // this tile's weight scales
+      if (G) {
+        const GTile g = gtile(t, p, gtab);
+        nt = g.nt;
+        arb = g.a_row0 / BM;
+        // a tile that does not start on a 128-row boundary spans two blocks
+        ablocks = ((g.a_row0 % BM) != 0 && arb + 1 < p.a_rowblocks) ? 2 : 1;
+        wsf += static_cast<long long>(g.e) * p.w_sf_bytes;
+      } else {
+        tile_coords(t, p, mt, nt);
+        arb = mt;
+      }
       const int rb0 = nt * BN / 128;
       const int wblocks = min(T::SF_BLOCKS, p.w_rowblocks - rb0);
       for (int kb = kb0; kb < kb1; ++kb) {
@@ -276,13 +387,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int cb0 = kb * kAtomsPerStage;
           const int atoms = min(kAtomsPerStage, p.ncb - cb0);
           const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
-          mbar_expect_tx(&sf_loaded[stage], sf_bytes * (1 + wblocks));
-          bulk_load(sSFA + stage * SFA_STAGE,
-                    p.a_scales + (static_cast<long long>(mt) * p.ncb + cb0) * 512, sf_bytes,
-                    &sf_loaded[stage]);
+          mbar_expect_tx(&sf_loaded[stage], sf_bytes * (ablocks + wblocks));
+          for (int i = 0; i < ablocks; ++i)
+            bulk_load(sSFA + stage * SFA_STAGE + i * kAtomsPerStage * 512,
+                      p.a_scales + (static_cast<long long>(arb + i) * p.ncb + cb0) * 512, sf_bytes,
+                      &sf_loaded[stage]);
           for (int i = 0; i < wblocks; ++i)
             bulk_load(sSFB + stage * T::SFB_STAGE + i * 2048,
-                      p.w_scales + (static_cast<long long>(rb0 + i) * p.ncb + cb0) * 512, sf_bytes,
+                      wsf + (static_cast<long long>(rb0 + i) * p.ncb + cb0) * 512, sf_bytes,
                       &sf_loaded[stage]);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -361,7 +473,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t phase = 0;
     for (int t = t_first; t < n_tiles_total; t += t_stride) {
       int mt, nt;
-      tile_coords(t, p, mt, nt);
+      // G: where tile row i = lane + 32 j of this lane's four words sits in
+      // the stage's two A scale blocks (byte offset; -1 past the tensor)
+      int a_word[4] = {0, 0, 0, 0};
+      if (G) {
+        const GTile g = gtile(t, p, gtab);
+        nt = g.nt;
+        const int arb = g.a_row0 / BM;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = g.a_row0 + lane + 32 * j;
+          const int blk = r / BM - arb;
+          const int rr = r % BM;
+          a_word[j] = (r / BM < p.a_rowblocks)
+                          ? blk * kAtomsPerStage * 512 + (rr & 31) * 16 + (rr >> 5) * 4
+                          : -1;
+        }
+      } else {
+        tile_coords(t, p, mt, nt);
+      }
       // BN = 64: the tile is rows 64 (nt & 1) .. +63 of its scale block,
       // words 2 (nt & 1) and 2 (nt & 1) + 1 of each 16-byte atom row
       const int half = (BN == 64) ? (nt & 1) : 0;
@@ -380,8 +510,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint32_t va[4 * kAtomsPerStage], vb[4 * T::SF_BLOCKS * kAtomsPerStage];
 #pragma unroll
           for (int a = 0; a < kAtomsPerStage; ++a) {
-            const uint4 x = lds128(sfa_s + a * 512);
-            va[4 * a + 0] = x.x; va[4 * a + 1] = x.y; va[4 * a + 2] = x.z; va[4 * a + 3] = x.w;
+            if (G) {
+              const uint32_t base = smem_u32(sSFA + stage * SFA_STAGE) + a * 512;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) va[4 * a + j] = a_word[j] >= 0 ? lds32(base + a_word[j]) : 0u;
+            } else {
+              const uint4 x = lds128(sfa_s + a * 512);
+              va[4 * a + 0] = x.x; va[4 * a + 1] = x.y; va[4 * a + 2] = x.z; va[4 * a + 3] = x.w;
+            }
 #pragma unroll
             for (int rb = 0; rb < T::SF_BLOCKS; ++rb) {
               const uint4 y = lds128(sfb_s + rb * 2048 + a * 512);
@@ -426,17 +562,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
       int it = 0;
       for (int t = t_first; t < n_tiles_total; t += t_stride, ++it) {
-        int mt, nt;
-        tile_coords(t, p, mt, nt);
+        int mt, nt, row, row_end = p.M;
+        if (G) {
+          const GTile g = gtile(t, p, gtab);
+          nt = g.nt;
+          row = g.a_row0 + quarter * 32 + lane;
+          row_end = g.a_row_end;
+          if (FMT == 0) alpha = __fmul_rn(*p.g_a, p.g_w[g.e]);
+        } else {
+          tile_coords(t, p, mt, nt);
+          row = mt * BM + quarter * 32 + lane;
+        }
         // warp-uniform outcome: tcgen05.ld below needs all 32 lanes
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag,
                                                p.watchdog, WD_EPILOGUE)))
           break;
         tc_fence_after();
-        const int row = mt * BM + quarter * 32 + lane;
-        const bool row_ok = row < p.M;
+        const bool row_ok = row < row_end;
         const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL;
-        if (!OUT_F32) {
+        if (OUT != 1) {
           // bf16: the whole row fits in registers once packed, so the
           // accumulator is released before any global store is issued
           uint32_t packed[BN / 2];
@@ -456,7 +600,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(acc_empty);
-          if (row_ok) {
+          if (OUT >= 2) {
+            const bool pad = p.qo.layout == 0 && !row_ok && row < (p.M + 127) / 128 * 128;
+            quant_out_row<BN, OUT - 2>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N);
+          }
+          if (row_ok && (OUT == 0 || p.C != nullptr)) {
             uint16_t* out = static_cast<uint16_t*>(p.C) + static_cast<long long>(row) * p.ldc;
 #pragma unroll
             for (int v = 0; v < BN / 8; ++v) {
@@ -575,7 +723,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] = (src == 0) ? x[i] : __fadd_rn(acc[i], x[i]);
           }
-          store8<OUT_F32>(p.C, (static_cast<long long>(mt) * BM + lo + lr) * p.ldc + nt * BN + 8 * g,
+          store8<OUT == 1>(p.C, (static_cast<long long>(mt) * BM + lo + lr) * p.ldc + nt * BN + 8 * g,
                           alpha, acc);
         }
       }
@@ -641,14 +789,27 @@ bool make_bf16_out_map(CUtensorMap* m, void* C, long long rows, int cols, int ld
   return r == CUDA_SUCCESS;
 }
 
+bool make_f32_out_map(CUtensorMap* m, void* C, long long rows, int cols, int ldc, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldc) * 4};
+  cuuint32_t box[2] = {32, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, C, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
-template <int FMT, int OUT_F32, int BN>
+template <int FMT, int OUT, int BN, int G = 0>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const Params& p, int grid,
                          cudaStream_t s) {
-  auto kern = gemm_kernel<FMT, OUT_F32, BN>;
+  auto kern = gemm_kernel<FMT, OUT, BN, G>;
   cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<BN>::SMEM);
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<BN, G>::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
@@ -665,7 +826,7 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const Par
   }
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = Tile<BN>::SMEM;
+  cfg.dynamicSmemBytes = Tile<BN, G>::SMEM;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = na;
@@ -723,11 +884,12 @@ cudaError_t launch_bn(const GemmArgs& a, Params p, int splits, cudaStream_t s) {
   p.k_per = (p.k_steps + splits - 1) / splits;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = (splits > 1) ? tiles * splits : std::max(1, std::min(tiles, sms));
-  if (a.fmt == 0)
-    return a.out_f32 ? launch_typed<0, 1, BN>(ma, mw, p, grid, s)
-                     : launch_typed<0, 0, BN>(ma, mw, p, grid, s);
-  return a.out_f32 ? launch_typed<1, 1, BN>(ma, mw, p, grid, s)
-                   : launch_typed<1, 0, BN>(ma, mw, p, grid, s);
+  using L = cudaError_t (*)(const CUtensorMap&, const CUtensorMap&, const Params&, int,
+                            cudaStream_t);
+  static const L table[2][4] = {
+      {launch_typed<0, 0, BN>, launch_typed<0, 1, BN>, launch_typed<0, 2, BN>, launch_typed<0, 3, BN>},
+      {launch_typed<1, 0, BN>, launch_typed<1, 1, BN>, launch_typed<1, 2, BN>, launch_typed<1, 3, BN>}};
+  return table[a.fmt != 0][a.out_mode](ma, mw, p, grid, s);
 }
 
 }  // namespace
@@ -756,13 +918,58 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   p.w_rowblocks = (a.N + 127) / 128;
   p.watchdog = watchdog_ptr();
   if (!p.watchdog) return cudaErrorInvalidSymbol;
-  const Shape sh = choose_shape(p.m_tiles, a.N, p.k_steps, sms, max_clusters_bn);
+  p.qo = a.qo;
+  // the FP4-emitting epilogue quantizes whole rows of a tile: no K split
+  const Shape sh = choose_shape(p.m_tiles, a.N, p.k_steps, sms, max_clusters_bn, a.out_mode < 2);
   if (sh.bn == 64) return launch_bn<64>(a, p, sh.splits, s);
   if (sh.bn == 128) return launch_bn<128>(a, p, sh.splits, s);
   return launch_bn<256>(a, p, sh.splits, s);
 }
 
-cudaError_t gemm_plan(int M, int N, int K, int max_sms, int* tile_m, int* tile_n, int* splits) {
+cudaError_t launch_gemm_grouped(const GroupedArgs& a, cudaStream_t s) {
+  const int sms = gemm_sms(a.max_sms);
+  Params p{};
+  p.a_scales = a.a_scales;
+  p.w_scales = a.w_scales;
+  p.g_a = a.g_a;
+  p.g_w = a.g_w;
+  p.C = a.C;
+  p.ldc = a.ldc;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  // M tiles of all groups together: at most one partial tile per group more
+  // than the rows alone need
+  p.m_tiles = (a.M + BM - 1) / BM + a.E;
+  p.k_steps = (a.K + BK - 1) / BK;
+  p.ncb = ncb_of(nsf_of(a.K, a.fmt));
+  p.w_rowblocks = (a.N + 127) / 128;
+  p.watchdog = watchdog_ptr();
+  if (!p.watchdog) return cudaErrorInvalidSymbol;
+  p.offsets = a.offsets;
+  p.E = a.E;
+  p.w_sf_bytes = static_cast<long long>(p.w_rowblocks) * p.ncb * 512;
+  p.a_rowblocks = (a.M + BM - 1) / BM;
+  p.splits = 1;
+  p.k_per = p.k_steps;
+  // 128 x 128 tiles with all of K (no split): the two A scale blocks a
+  // stage may need leave no room for a 256-wide tile's ring
+  const int bn = 128;
+  CUtensorMap ma, mw;
+  if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM)) return cudaErrorInvalidValue;
+  if (!make_code_map(&mw, a.w_codes, static_cast<long long>(a.E) * a.N, a.K, bn))
+    return cudaErrorInvalidValue;
+  p.n_tiles = (a.N + bn - 1) / bn;
+  const long long upper = static_cast<long long>(p.m_tiles) * p.n_tiles;
+  const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(upper, sms)));
+  return a.fmt == 0 ? (a.out_f32 ? launch_typed<0, 1, 128, 1>(ma, mw, p, grid, s)
+                                 : launch_typed<0, 0, 128, 1>(ma, mw, p, grid, s))
+                    : (a.out_f32 ? launch_typed<1, 1, 128, 1>(ma, mw, p, grid, s)
+                                 : launch_typed<1, 0, 128, 1>(ma, mw, p, grid, s));
+}
+
+cudaError_t gemm_plan(int M, int N, int K, int max_sms, int* tile_m, int* tile_n, int* splits,
+                      bool allow_split) {
   const int sms = gemm_sms(max_sms);
   if (sms <= 0) return cudaErrorNoDevice;
   if (takes_pair(M, N, sms)) {
@@ -771,7 +978,8 @@ cudaError_t gemm_plan(int M, int N, int K, int max_sms, int* tile_m, int* tile_n
     *splits = 1;
     return cudaSuccess;
   }
-  const Shape sh = choose_shape((M + BM - 1) / BM, N, (K + BK - 1) / BK, sms, max_clusters_bn);
+  const Shape sh = choose_shape((M + BM - 1) / BM, N, (K + BK - 1) / BK, sms, max_clusters_bn,
+                                allow_split);
   *tile_m = BM;
   *tile_n = sh.bn;
   *splits = sh.splits;

@@ -48,6 +48,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "out_quant.cuh"
 #include "ptx.cuh"
 
 namespace fp4 {
@@ -95,6 +96,7 @@ struct Params {
   int a_rowblocks;        // ceil(M / 128)
   int w_rowblocks;        // ceil(N / 128)
   unsigned* watchdog;
+  QuantOut qo;            // OUT >= 2: the emitted FP4 activation (C optional)
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int& nt) {
@@ -107,7 +109,9 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int
   nt = within / gsize;
 }
 
-template <int FMT, int OUT_F32>
+// OUT: 0 = bf16 C, 1 = fp32 C, 2 / 3 = C quantized to NVFP4 / MXFP4
+// (out_quant.cuh), with the bf16 C stored as well when p.C is not null.
+template <int FMT, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_w,
@@ -151,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_w);
-    if (!OUT_F32) prefetch_tensormap(&tm_c);
+    if (OUT <= 1 || p.C != nullptr) prefetch_tensormap(&tm_c);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -391,6 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (FMT == 0) alpha = __fmul_rn(*p.g_a, *p.g_w);
     const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
     uint8_t* sOutW = sOut + (warp - 2) * 2 * OUT_BUF;
+    QuantOutG qg{};
+    if (OUT >= 2) qg = quant_out_g(p.qo);
     int it = 0;
     for (int t = first; t < n_tiles_total; t += stride, ++it) {
       int mt, nt;
@@ -404,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = mt * BM + static_cast<int>(rank) * HALF + quarter * 32 + lane;
       const bool row_ok = row < p.M;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL;
-      if (!OUT_F32) {
+      if (OUT != 1) {
         uint32_t packed[BN / 2];
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
@@ -431,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // buffers and 64-column TMA stores (rows past M and columns past N
         // are clipped by the store)
         const int row0 = mt * BM + static_cast<int>(rank) * HALF + quarter * 32;
-        if (row0 < p.M) {
+        if (row0 < p.M && (OUT == 0 || p.C != nullptr)) {
 #pragma unroll
           for (int c = 0; c < BN / 64; ++c) {
             const int n0 = nt * BN + 64 * c;
@@ -455,7 +461,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        if (OUT >= 2) {
+          const bool pad = p.qo.layout == 0 && !row_ok && row < p.a_rowblocks * HALF;
+          quant_out_row<BN, OUT - 2>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N);
+        }
       } else {
+        // fp32: 32-column chunks leave through the warp's two swizzled
+        // buffers (32 rows x 128 bytes each) and TMA stores (clipped at M
+        // and N), so that the warp's writes are whole 128-byte rows issued
+        // by the copy engine instead of 32 scattered 16-byte stores per
+        // instruction; the accumulator is released after its last chunk is
+        // read
+        const int row0 = mt * BM + static_cast<int>(rank) * HALF + quarter * 32;
+#pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
           FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
@@ -471,24 +489,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           const int n0 = nt * BN + c * 32;
-          if (!row_ok || n0 >= p.N) continue;
-          float* out = static_cast<float*>(p.C) + static_cast<long long>(row) * p.ldc + n0;
+          if (row0 >= p.M || n0 >= p.N) continue;   // warp-uniform
+          uint8_t* buf = sOutW + (c & 1) * OUT_BUF;
+          // the buffer's previous store must have finished reading it
+          if (lane == 0) bulk_wait_read_1();
+          __syncwarp();
+          const uint32_t rowaddr = smem_u32(buf) + lane * 128;
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            if (n0 + 4 * v < p.N) {
-              float4 o;
-              o.x = __fmul_rn(alpha, __uint_as_float(r[4 * v + 0]));
-              o.y = __fmul_rn(alpha, __uint_as_float(r[4 * v + 1]));
-              o.z = __fmul_rn(alpha, __uint_as_float(r[4 * v + 2]));
-              o.w = __fmul_rn(alpha, __uint_as_float(r[4 * v + 3]));
-              *reinterpret_cast<float4*>(out + 4 * v) = o;
-            }
+          for (int j = 0; j < 8; ++j)
+            sts128(rowaddr + ((j ^ (lane & 7)) << 4),
+                   __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[4 * j + 0]))),
+                   __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[4 * j + 1]))),
+                   __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[4 * j + 2]))),
+                   __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[4 * j + 3]))));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_c, buf, n0, row0);
+            bulk_commit();
           }
         }
       }
     }
     // every TMA store of this warp has landed before the CTA goes away
-    if (!OUT_F32 && lane == 0) bulk_wait_all();
+    if (lane == 0) bulk_wait_all();
     __syncwarp();
   }
 
@@ -505,10 +529,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------ host side
 
-template <int FMT, int OUT_F32>
+template <int FMT, int OUT>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc,
                          const Params& p, int tiles, int max_sms, cudaStream_t s) {
-  auto kern = gemm_pair_kernel<FMT, OUT_F32>;
+  auto kern = gemm_pair_kernel<FMT, OUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -549,9 +573,10 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
   CUtensorMap ma, mw, mc;
   if (!make_code_map(&ma, a.a_codes, a.M, a.K, HALF)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, a.w_codes, a.N, a.K, HALF)) return cudaErrorInvalidValue;
-  if (a.out_f32)
-    mc = ma;   // unused by the fp32 epilogue
-  else if (!make_bf16_out_map(&mc, a.C, a.M, a.N, a.ldc, 32))
+  if (a.out_mode >= 2 && !a.C)
+    mc = ma;   // unused: no bf16 C beside the FP4 output
+  else if (a.out_mode == 1 ? !make_f32_out_map(&mc, a.C, a.M, a.N, a.ldc, 32)
+                           : !make_bf16_out_map(&mc, a.C, a.M, a.N, a.ldc, 32))
     return cudaErrorInvalidValue;
   Params p;
   p.a_scales = a.a_scales;
@@ -571,12 +596,14 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
   p.w_rowblocks = (a.N + HALF - 1) / HALF;
   p.watchdog = watchdog_ptr();
   if (!p.watchdog) return cudaErrorInvalidSymbol;
+  p.qo = a.qo;
   const int tiles = p.m_tiles * p.n_tiles;
-  if (a.fmt == 0)
-    return a.out_f32 ? launch_typed<0, 1>(ma, mw, mc, p, tiles, a.max_sms, s)
-                     : launch_typed<0, 0>(ma, mw, mc, p, tiles, a.max_sms, s);
-  return a.out_f32 ? launch_typed<1, 1>(ma, mw, mc, p, tiles, a.max_sms, s)
-                   : launch_typed<1, 0>(ma, mw, mc, p, tiles, a.max_sms, s);
+  using L = cudaError_t (*)(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                            const Params&, int, int, cudaStream_t);
+  static const L table[2][4] = {
+      {launch_typed<0, 0>, launch_typed<0, 1>, launch_typed<0, 2>, launch_typed<0, 3>},
+      {launch_typed<1, 0>, launch_typed<1, 1>, launch_typed<1, 2>, launch_typed<1, 3>}};
+  return table[a.fmt != 0][a.out_mode](ma, mw, mc, p, tiles, a.max_sms, s);
 }
 
 }  // namespace fp4

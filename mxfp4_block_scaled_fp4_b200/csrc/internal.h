@@ -8,6 +8,7 @@
 namespace fp4 {
 
 constexpr int kAmaxSlots = 1024;   // partial maxima of the global-scale reduction
+constexpr int kGroupedMaxGroups = 256;   // groups (experts) of one fp4_gemm_grouped call
 
 // Workspace bytes the activation quantizer needs (the DYNAMIC reduction's
 // partial maxima); one rule for every entry point that quantizes.
@@ -32,6 +33,10 @@ inline long long rows_pad128(long long rows) { return (rows + 127) / 128 * 128; 
 // predecessor before reading their input).
 cudaError_t launch_amax(const void* x, long long n, unsigned* partial, int* n_used,
                         cudaStream_t s, bool pdl = false);
+// The same over the rotated values of a [rows, K] tensor (rot = 16 or 32,
+// times scale): one partial maximum per CTA as binary32 magnitude bits.
+cudaError_t launch_amax_rot(const void* x, long long rows, int K, int rot, float scale,
+                            unsigned* partial, int* n_used, cudaStream_t s, bool pdl = false);
 
 struct QuantArgs {
   const void* x;        // bf16 [rows, K]
@@ -60,6 +65,13 @@ struct QuantArgs {
   // The status word a non-finite DYNAMIC maximum is reported in (set by
   // launch_quantize when null).
   unsigned* status = nullptr;
+  // Online rotation: 0 (none), 16 or 32 (block-diagonal Walsh-Hadamard of
+  // that order along K, then a multiply by rot_scale = 2^-shift).  The
+  // partial maxima of a rotated tensor's amax pass are binary32 bits.
+  int rot = 0;
+  float rot_scale = 1.0f;
+  // MXFP4 scale rule: 0 = OCP (floor(log2 amax) - 2), 1 = overflow-aware.
+  int rule = 0;
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl = false);
 
@@ -78,22 +90,44 @@ constexpr long long kSelfAmaxBytes = 32 << 10;
 // bandwidth, and two launches cost ~5 us whatever the size.)
 cudaError_t launch_quantize_act(QuantArgs a, unsigned* partial, cudaStream_t s);
 
+}  // namespace fp4
+#include "out_quant.cuh"
+namespace fp4 {
+
 struct GemmArgs {
   const uint8_t* a_codes; const uint8_t* a_scales; const float* g_a;
   const uint8_t* w_codes; const uint8_t* w_scales; const float* g_w;
   int M, N, K, fmt;
-  void* C; int ldc; int out_f32;
+  void* C; int ldc;
+  int out_mode;         // 0 bf16 C, 1 fp32 C, 2 / 3 NVFP4 / MXFP4 activation (+ bf16 C if C)
   int max_sms;          // SMs the launch shape is chosen for, 0 = the device's
+  QuantOut qo;          // out_mode 2, 3
 };
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s);
 // The shape launch_gemm takes: tile rows x columns, CTAs per tile along K.
-cudaError_t gemm_plan(int M, int N, int K, int max_sms, int* tile_m, int* tile_n, int* splits);
+// allow_split = false: the shape the FP4-emitting epilogue takes (no K split).
+cudaError_t gemm_plan(int M, int N, int K, int max_sms, int* tile_m, int* tile_n, int* splits,
+                      bool allow_split = true);
 // The SMs a GEMM's launch shape is chosen for: max_sms when 0 < max_sms <
 // the device's count, else the device's.
 int gemm_sms(int max_sms);
 // The CTA-pair kernel (256 x 256 tiles); launch_gemm takes it for M > 128
 // when its tiles keep at least half the SMs busy.
 cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s);
+
+// The grouped (mixture-of-experts) GEMM: group e multiplies rows
+// [offsets[e], offsets[e+1]) of A by weight e of the stacked W (E x [N, K],
+// per-expert scale blocks of w_sf_bytes, global scales g_w[e]); offsets is
+// a device array of E + 1 ints.
+struct GroupedArgs {
+  const uint8_t* a_codes; const uint8_t* a_scales; const float* g_a;
+  const uint8_t* w_codes; const uint8_t* w_scales; const float* g_w;
+  const int* offsets;
+  int E, M, N, K, fmt;
+  void* C; int ldc; int out_f32;
+  int max_sms;
+};
+cudaError_t launch_gemm_grouped(const GroupedArgs& a, cudaStream_t s);
 
 // Tensor map of packed FP4 codes [rows, K/2] bytes as a 2-D uint8 tensor:
 // box of 128 bytes of K by box_rows rows, 128-byte swizzle, out-of-range
@@ -103,6 +137,8 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, long long rows, int K, i
 // Tensor map of a bf16 output C [rows, cols] with row pitch ldc elements:
 // box of 64 columns (128 bytes) by box_rows rows, 128-byte swizzle.
 bool make_bf16_out_map(CUtensorMap* m, void* C, long long rows, int cols, int ldc, int box_rows);
+// The same for an fp32 C: box of 32 columns (128 bytes) by box_rows rows.
+bool make_f32_out_map(CUtensorMap* m, void* C, long long rows, int cols, int ldc, int box_rows);
 
 struct FusedArgs {
   const void* a;        // bf16 [M, K]
@@ -112,6 +148,9 @@ struct FusedArgs {
   void* C; int ldc; int out_f32;
   void* ws; size_t ws_bytes;
   int max_sms;          // SMs the launch shape is chosen for, 0 = the device's
+  int rot = 0;          // activation rotation (QuantArgs::rot), its scale, MXFP4 rule
+  float rot_scale = 1.0f;
+  int rule = 0;
 };
 size_t fused_workspace_bytes(int M, int N, int K, int fmt);
 // Shapes the fused path takes: 1 <= M <= 32 and K up to 8 slices of 8192.

@@ -29,8 +29,11 @@ inline bool takes_pair(int M, int N, int sms) {
 // 256-wide tiles, or clusters on nearly every SM, they measured slower
 // than every alternative).  max_clusters(bn, S): clusters of S CTAs of the
 // bn-wide kernel the device can hold at once (0 when unknown).
+// allow_split = false keeps S = 1 (the epilogue that emits FP4 codes needs
+// whole rows of a tile in one CTA).
 template <typename MaxClusters>
-Shape choose_shape(int m_tiles, int N, int k_steps, int sms, MaxClusters max_clusters) {
+Shape choose_shape(int m_tiles, int N, int k_steps, int sms, MaxClusters max_clusters,
+                   bool allow_split = true) {
   Shape best;
   double best_t = 1e30;
   for (int bn : {256, 128, 64}) {
@@ -43,7 +46,8 @@ Shape choose_shape(int m_tiles, int N, int k_steps, int sms, MaxClusters max_clu
         const int waves = (tiles + sms - 1) / sms;
         t = waves * (128.0 + bn) * k_per * 144.0 / 112.0;
       } else {
-        if (bn == 256 || (k_steps + k_per - 1) / k_per != S || tiles * S * 100 > sms * 85)
+        if (!allow_split || bn == 256 || (k_steps + k_per - 1) / k_per != S ||
+            tiles * S * 100 > sms * 85)
           continue;
         if (tiles > max_clusters(bn, S)) continue;
         t = (128.0 + bn) * k_per * 144.0 / 112.0 + 1500.0 +

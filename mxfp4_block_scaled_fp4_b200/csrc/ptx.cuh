@@ -27,6 +27,9 @@ static_assert(WD_NONFINITE == FP4_STATUS_NONFINITE_BIT, "status bit of fp4.h");
 // is Inf (0x7F80) or NaN.
 constexpr unsigned kBf16MaxFinite = 0x7F7Fu;
 
+// The largest finite binary32 magnitude pattern (rotated tensors' maxima).
+constexpr unsigned kF32MaxFinite = 0x7F7FFFFFu;
+
 // A DYNAMIC global-scale reduction's final maximum (bf16 magnitude bits):
 // a non-finite input is reported in the status word and the maximum is
 // clamped to the largest finite bf16, so g stays finite.
@@ -34,6 +37,15 @@ __device__ __forceinline__ unsigned amax_checked(unsigned m, unsigned* wd) {
   if (m > kBf16MaxFinite) {
     atomicOr(wd, WD_NONFINITE);
     return kBf16MaxFinite;
+  }
+  return m;
+}
+
+// The same for a maximum in binary32 magnitude bits (rotated tensors).
+__device__ __forceinline__ unsigned amax_checked_f32(unsigned m, unsigned* wd) {
+  if (m > kF32MaxFinite) {
+    atomicOr(wd, WD_NONFINITE);
+    return kF32MaxFinite;
   }
   return m;
 }
@@ -434,6 +446,12 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* v) {
 }
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t saddr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t saddr) {

@@ -45,26 +45,43 @@ __device__ __forceinline__ long long mma_scale_offset(long long r, int c, int nc
 // caller's value (STATIC).  g = amax / 2688, 1 for an all-zero tensor.
 // self_amax: the maximum over the whole tensor x (n_vec 16-byte vectors)
 // instead of the partial maxima (small tensors; 4 loads in flight a thread).
+// With a rotation (ROT = 16 or 32) the maximum is over the rotated values
+// and the partial maxima are binary32 magnitude bits; without, bf16 bits.
 // A non-finite input is reported in `status` and the maximum clamped to the
-// largest finite bf16 (amax_checked), so g stays finite.
+// largest finite value (amax_checked), so g stays finite.
+template <int ROT>
 __device__ float global_scale(int dynamic, const float* g, const unsigned* partial,
                               int n_partial, int self_amax, const uint4* x, long long n_vec,
-                              unsigned* status) {
+                              unsigned* status, float rot_scale) {
   if (!dynamic) return *g;
   __shared__ unsigned red[kThreads / 32];
   unsigned m = 0;
   if (self_amax) {
-    for (long long i = threadIdx.x; i < n_vec; i += 4 * blockDim.x) {
-      uint4 v[4];
+    if (ROT == 0) {
+      for (long long i = threadIdx.x; i < n_vec; i += 4 * blockDim.x) {
+        uint4 v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const long long k = i + j * blockDim.x;
-        v[j] = (k < n_vec) ? ld_stream(x + k) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < 4; ++j) {
+          const long long k = i + j * blockDim.x;
+          v[j] = (k < n_vec) ? ld_stream(x + k) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m = max_u16x2(m, mag_max8(v[j]));
       }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) m = max_u16x2(m, mag_max8(v[j]));
+      m = fold_u16x2(m);
+    } else {
+      // units of 16 values; whole warps iterate together (lane pairs)
+      const long long n_units = n_vec / 2;
+      for (long long base = 0; base < n_units; base += blockDim.x) {
+        const long long u = base + threadIdx.x;
+        const uint4 p = (u < n_units) ? ld_stream(x + 2 * u) : make_uint4(0, 0, 0, 0);
+        const uint4 q = (u < n_units) ? ld_stream(x + 2 * u + 1) : make_uint4(0, 0, 0, 0);
+        float f[16];
+        unpack16(p, q, f);
+        rotate_unit<ROT>(f, rot_scale, (threadIdx.x & 1) != 0);
+        m = max(m, mag_max16(f));
+      }
     }
-    m = fold_u16x2(m);
   } else {
     for (int i = threadIdx.x; i < n_partial; i += blockDim.x) m = max(m, partial[i]);
   }
@@ -73,10 +90,17 @@ __device__ float global_scale(int dynamic, const float* g, const unsigned* parti
   __syncthreads();
   m = 0;
   for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) m = max(m, red[i]);
-  // one CTA reports a non-finite input; every CTA clamps alike
-  if (m > kBf16MaxFinite) m = (blockIdx.x == 0 && threadIdx.x == 0) ? amax_checked(m, status)
-                                                                      : kBf16MaxFinite;
-  const float amax = __uint_as_float(m << 16);
+  float amax;
+  if (ROT == 0) {
+    // one CTA reports a non-finite input; every CTA clamps alike
+    if (m > kBf16MaxFinite) m = (blockIdx.x == 0 && threadIdx.x == 0) ? amax_checked(m, status)
+                                                                        : kBf16MaxFinite;
+    amax = __uint_as_float(m << 16);
+  } else {
+    if (m > kF32MaxFinite) m = (blockIdx.x == 0 && threadIdx.x == 0) ? amax_checked_f32(m, status)
+                                                                       : kF32MaxFinite;
+    amax = __uint_as_float(m);
+  }
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
 
@@ -121,6 +145,51 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const uint4* __restri
   }
 }
 
+// The amax pass over rotated values: warps take slabs of 4 x 32 units of 16
+// values (every lane issues its 8 loads first), rotate each unit and keep
+// the largest magnitude (binary32 bits).
+template <int ROT>
+__global__ void __launch_bounds__(kThreads, 4) amax_rot_kernel(const uint4* __restrict__ x,
+                                                               long long n_units, float scale,
+                                                               unsigned* __restrict__ partial) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const long long n_slabs = (n_units + 127) / 128;
+  const long long gwarp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  unsigned m = 0;
+  for (long long t = gwarp; t < n_slabs; t += nwarps) {
+    uint4 v[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long long u = t * 128 + j * 32 + lane;
+      if (u < n_units) {
+        v[j][0] = ld_stream(x + 2 * u);
+        v[j][1] = ld_stream(x + 2 * u + 1);
+      } else {
+        v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float f[16];
+      unpack16(v[j][0], v[j][1], f);
+      rotate_unit<ROT>(f, scale, (lane & 1) != 0);
+      m = max(m, mag_max16(f));
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ unsigned red[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned r = 0;
+    for (int w = 0; w < kThreads / 32; ++w) r = max(r, red[w]);
+    partial[blockIdx.x] = r;
+  }
+}
+
 // -------------------------------------------------------- quantize pass
 
 // n / d for 32-bit n by multiply-high (Granlund & Montgomery, "Division by
@@ -138,7 +207,7 @@ __device__ __forceinline__ unsigned fast_div(unsigned n, FastDiv f) {
 // Units [u_begin, u_end) in slabs of 4 x 32 consecutive units: warp w of
 // nwarps takes slabs w, w + nwarps, ... (from the end when `reverse`), and
 // every lane issues its 8 loads (4 units x 32 bytes) before computing.
-template <int FMT, int LAYOUT>
+template <int FMT, int LAYOUT, int ROT>
 __device__ __forceinline__ void quantize_units(const QuantArgs& a, long long u_begin,
                                                long long u_end, long long w, long long nwarps,
                                                bool reverse, int upr, FastDiv upr_div, int nsf,
@@ -167,19 +236,37 @@ __device__ __forceinline__ void quantize_units(const QuantArgs& a, long long u_b
     for (int j = 0; j < 4; ++j) {
       const long long u = u_begin + slab * 128 + j * 32 + lane;
       const uint4 p = xs[j][0], q = xs[j][1];
-      unsigned m = fold_u16x2(max_u16x2(mag_max8(p), mag_max8(q)));
       unsigned sbyte;
       uint2 packed;
       float r;
-      if (FMT == 0) {
-        sbyte = nvfp4_scale_byte(m, six_g, y6, fast_b);
-        r = r_tab[sbyte & 127u];
-        packed = (r == 0.0f) ? make_uint2(0, 0)
-                             : make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
+      if (ROT == 0) {
+        unsigned m = fold_u16x2(max_u16x2(mag_max8(p), mag_max8(q)));
+        if (FMT == 0) {
+          sbyte = nvfp4_scale_byte(m, six_g, y6, fast_b);
+          r = r_tab[sbyte & 127u];
+          packed = (r == 0.0f) ? make_uint2(0, 0)
+                               : make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
+        } else {
+          m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));   // 32-value block = lane pair
+          sbyte = mxfp4_scale_f32(m << 16, a.rule, &r);
+          packed = make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
+        }
       } else {
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));   // 32-value block = lane pair
-        sbyte = mxfp4_scale(m, &r);
-        packed = make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
+        // the unit's rotated values (a 32-value rotation pairs lanes 2i, 2i+1:
+        // their units are the two halves of one 32-value block)
+        float f[16];
+        unpack16(p, q, f);
+        rotate_unit<ROT>(f, a.rot_scale, (lane & 1) != 0);
+        unsigned m = mag_max16(f);
+        if (FMT == 0) {
+          sbyte = nvfp4_scale_byte_f32(m, six_g, y6, fast_b);
+          r = r_tab[sbyte & 127u];
+          packed = (r == 0.0f) ? make_uint2(0, 0) : make_uint2(quant8_f32(f, r), quant8_f32(f + 8, r));
+        } else {
+          m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+          sbyte = mxfp4_scale_f32(m, a.rule, &r);
+          packed = make_uint2(quant8_f32(f, r), quant8_f32(f + 8, r));
+        }
       }
       if (u < u_end) {
         codes[u] = packed;
@@ -220,15 +307,16 @@ __device__ __forceinline__ void zero_mma_padding(const QuantArgs& a, long long p
 
 // The full-chip quantize pass.  With a DYNAMIC global scale the slabs are
 // walked from the end, so the first ones are still in L2 from the amax pass.
-template <int FMT, int LAYOUT>
+template <int FMT, int LAYOUT, int ROT>
 __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long long units,
                                                                int upr, FastDiv upr_div, int nsf,
                                                                int ncb, long long pad_a,
                                                                long long pad_b) {
   if (a.release_early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const float g = (FMT == 0) ? global_scale(a.dynamic, a.g, a.partial, a.n_partial, a.self_amax,
-                                            static_cast<const uint4*>(a.x), units * 2, a.status)
+  const float g = (FMT == 0) ? global_scale<ROT>(a.dynamic, a.g, a.partial, a.n_partial,
+                                                 a.self_amax, static_cast<const uint4*>(a.x),
+                                                 units * 2, a.status, a.rot_scale)
                              : 1.0f;
   if (FMT == 0 && a.dynamic && blockIdx.x == 0 && threadIdx.x == 0) *a.g = g;
   const float six_g = __fmul_rn(6.0f, g);
@@ -242,8 +330,8 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long
   }
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long gwarp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  quantize_units<FMT, LAYOUT>(a, 0, units, gwarp, stride >> 5, a.dynamic != 0, upr, upr_div, nsf,
-                              ncb, six_g, y6, fast_b, r_tab);
+  quantize_units<FMT, LAYOUT, ROT>(a, 0, units, gwarp, stride >> 5, a.dynamic != 0, upr, upr_div,
+                                   nsf, ncb, six_g, y6, fast_b, r_tab);
   if (LAYOUT == 0)
     zero_mma_padding(a, pad_a, pad_b, nsf, ncb,
                      static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x, stride);
@@ -280,6 +368,19 @@ cudaError_t launch_k(void (*k)(Args...), int blocks, bool pdl, cudaStream_t s, A
   return cudaLaunchKernelEx(&cfg, k, args...);
 }
 }  // namespace
+
+cudaError_t launch_amax_rot(const void* x, long long rows, int K, int rot, float scale,
+                            unsigned* partial, int* n_used, cudaStream_t s, bool pdl) {
+  const long long n_units = rows * (K / 16);
+  long long want = (n_units + kThreads * 4 - 1) / (kThreads * 4);
+  int blocks = static_cast<int>(std::min<long long>(want, static_cast<long long>(sm_count()) * 4));
+  blocks = std::max(1, std::min(blocks, kAmaxSlots));
+  *n_used = blocks;
+  auto kern = (rot == 32) ? amax_rot_kernel<32> : amax_rot_kernel<16>;
+  const cudaError_t e = launch_k(kern, blocks, pdl, s, static_cast<const uint4*>(x), n_units,
+                                 scale, partial);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 cudaError_t launch_amax(const void* x, long long n, unsigned* partial, int* n_used,
                         cudaStream_t s, bool pdl) {
@@ -333,8 +434,16 @@ cudaError_t launch_quantize(const QuantArgs& a_in, cudaStream_t s, bool pdl) {
                                   (q.pad_a + q.pad_b + kThreads - 1) / kThreads);
   const int blocks = static_cast<int>(
       std::max<long long>(1, std::min<long long>(want, static_cast<long long>(sm_count()) * 4)));
-  auto kern = (a.fmt == 0) ? (a.layout == 0 ? quantize_kernel<0, 0> : quantize_kernel<0, 1>)
-                           : (a.layout == 0 ? quantize_kernel<1, 0> : quantize_kernel<1, 1>);
+  using Kern = void (*)(QuantArgs, long long, int, FastDiv, int, int, long long, long long);
+  static const Kern table[3][2][2] = {
+      {{quantize_kernel<0, 0, 0>, quantize_kernel<0, 1, 0>},
+       {quantize_kernel<1, 0, 0>, quantize_kernel<1, 1, 0>}},
+      {{quantize_kernel<0, 0, 16>, quantize_kernel<0, 1, 16>},
+       {quantize_kernel<1, 0, 16>, quantize_kernel<1, 1, 16>}},
+      {{quantize_kernel<0, 0, 32>, quantize_kernel<0, 1, 32>},
+       {quantize_kernel<1, 0, 32>, quantize_kernel<1, 1, 32>}}};
+  const int ri = a.rot == 32 ? 2 : (a.rot == 16 ? 1 : 0);
+  const Kern kern = table[ri][a.fmt != 0][a.layout != 0];
   const cudaError_t e =
       launch_k(kern, blocks, pdl, s, a, q.units, q.upr, q.fd, q.nsf, q.ncb, q.pad_a, q.pad_b);
   if (e != cudaSuccess) return e;
@@ -348,7 +457,9 @@ cudaError_t launch_quantize_act(QuantArgs a, unsigned* partial, cudaStream_t s) 
   }
   if (a.dynamic) {
     int used = 0;
-    const cudaError_t e = launch_amax(a.x, a.rows * a.K, partial, &used, s, true);
+    const cudaError_t e =
+        a.rot ? launch_amax_rot(a.x, a.rows, a.K, a.rot, a.rot_scale, partial, &used, s, true)
+              : launch_amax(a.x, a.rows * a.K, partial, &used, s, true);
     if (e != cudaSuccess) return e;
     a.partial = partial;
     a.n_partial = used;

@@ -38,6 +38,21 @@ FP4_GLOBAL_STATIC = 1
 # fp4_out_t
 FP4_OUT_BF16 = 0
 FP4_OUT_F32 = 1
+# fp4_mx_rule_t
+FP4_MX_RULE_OCP = 0
+FP4_MX_RULE_OAS = 1
+
+
+class QuantOpts(ctypes.Structure):
+    """fp4_quant_opts_t: online rotation order (0, 16, 32) and MXFP4 rule."""
+    _fields_ = [("hadamard", ctypes.c_int), ("mx_rule", ctypes.c_int)]
+
+
+def opts(hadamard: int = 0, mx_rule: int = 0):
+    """A fp4_quant_opts_t by reference, or None when both are defaults."""
+    if not hadamard and not mx_rule:
+        return None
+    return ctypes.byref(QuantOpts(hadamard, mx_rule))
 
 
 class Fp4Error(RuntimeError):
@@ -61,8 +76,15 @@ SIGNATURES = {
     "fp4_workspace_bytes": (SZ, [I, I, I, I]),
     "fp4_quantize_act": (I, [P, I, I, I, I, I, FP, U8P, U8P, P, SZ, P]),
     "fp4_quantize_weights": (I, [P, I, I, I, U8P, U8P, FP, P, SZ, P]),
+    "fp4_quantize_act_ex": (I, [P, I, I, I, I, I, P, FP, U8P, U8P, P, SZ, P]),
+    "fp4_quantize_weights_ex": (I, [P, I, I, I, P, U8P, U8P, FP, P, SZ, P]),
+    "fp4_gemm_fused_ex": (I, [P, U8P, U8P, FP, I, I, I, I, I, P, FP, P, I, I, P, SZ, I, P]),
     "fp4_gemm": (I, [U8P, U8P, FP, U8P, U8P, FP, I, I, I, I, P, I, I, P, SZ, I, P]),
     "fp4_gemm_fused": (I, [P, U8P, U8P, FP, I, I, I, I, I, FP, P, I, I, P, SZ, I, P]),
+    "fp4_gemm_quant": (I, [U8P, U8P, FP, U8P, U8P, FP, I, I, I, I, I, I, P, FP, U8P, U8P, P, I,
+                           P, SZ, I, P]),
+    "fp4_gemm_grouped": (I, [U8P, U8P, FP, U8P, U8P, FP, P, I, I, I, I, I, P, I, I, P, SZ, I,
+                             P]),
     "fp4_gemm_plan": (I, [I, I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
     "fp4_quantize_act_noalloc": (I, [P, I, I, I, I, I, FP, U8P, U8P, P]),
     "fp4_device_status": (I, [ctypes.POINTER(ctypes.c_uint), P]),
@@ -121,6 +143,23 @@ def fp4_quantize_weights(w, N, K, fmt, codes, scales, g, ws, ws_bytes, stream):
     return _call("fp4_quantize_weights", w, N, K, fmt, codes, scales, g, ws, ws_bytes, stream)
 
 
+def fp4_quantize_act_ex(x, rows, K, fmt, layout, gmode, opts, g, codes, scales, ws, ws_bytes,
+                        stream):
+    return _call("fp4_quantize_act_ex", x, rows, K, fmt, layout, gmode, opts, g, codes, scales,
+                 ws, ws_bytes, stream)
+
+
+def fp4_quantize_weights_ex(w, N, K, fmt, opts, codes, scales, g, ws, ws_bytes, stream):
+    return _call("fp4_quantize_weights_ex", w, N, K, fmt, opts, codes, scales, g, ws, ws_bytes,
+                 stream)
+
+
+def fp4_gemm_fused_ex(a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, opts, g_a, C, ldc, out, ws,
+                      ws_bytes, max_sms, stream):
+    return _call("fp4_gemm_fused_ex", a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, opts, g_a,
+                 C, ldc, out, ws, ws_bytes, max_sms, stream)
+
+
 def fp4_gemm(a_codes, a_scales, g_a, w_codes, w_scales, g_w, M, N, K, fmt, C, ldc, out, ws,
              ws_bytes, max_sms, stream):
     return _call("fp4_gemm", a_codes, a_scales, g_a, w_codes, w_scales, g_w, M, N, K, fmt, C,
@@ -131,6 +170,20 @@ def fp4_gemm_fused(a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc, 
                    ws_bytes, max_sms, stream):
     return _call("fp4_gemm_fused", a, w_codes, w_scales, g_w, M, N, K, fmt, gmode, g_a, C, ldc,
                  out, ws, ws_bytes, max_sms, stream)
+
+
+def fp4_gemm_quant(a_codes, a_scales, g_a, w_codes, w_scales, g_w, M, N, K, fmt, out_fmt,
+                   out_layout, out_opts, g_out, out_codes, out_scales, C, ldc, ws, ws_bytes,
+                   max_sms, stream):
+    return _call("fp4_gemm_quant", a_codes, a_scales, g_a, w_codes, w_scales, g_w, M, N, K, fmt,
+                 out_fmt, out_layout, out_opts, g_out, out_codes, out_scales, C, ldc, ws,
+                 ws_bytes, max_sms, stream)
+
+
+def fp4_gemm_grouped(a_codes, a_scales, g_a, w_codes, w_scales, g_w, offsets, E, M, N, K, fmt,
+                     C, ldc, out, ws, ws_bytes, max_sms, stream):
+    return _call("fp4_gemm_grouped", a_codes, a_scales, g_a, w_codes, w_scales, g_w, offsets, E,
+                 M, N, K, fmt, C, ldc, out, ws, ws_bytes, max_sms, stream)
 
 
 def fp4_gemm_plan(M, N, K, fmt, max_sms, tile_m, tile_n, splits):

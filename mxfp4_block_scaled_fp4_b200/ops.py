@@ -56,14 +56,17 @@ class Quantized:
     layout: int
     rows: int
     K: int
+    hadamard: int = 0        # online rotation order (0, 16, 32)
+    mx_rule: int = 0         # MXFP4 scale rule (0 OCP, 1 overflow-aware)
 
 
 def quantize(x: torch.Tensor, fmt: int = NVFP4, layout: int = SCALES_MMA,
-             g: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> Quantized:
-    """fp4_quantize_act: DYNAMIC global scale when g is None, else STATIC g.
-    ws: scratch of at least fp4_workspace_bytes bytes; calls that may run
-    concurrently (other streams) need their own, else the shared per-device
-    buffer is used."""
+             g: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+             hadamard: int = 0, mx_rule: int = 0) -> Quantized:
+    """fp4_quantize_act (fp4_quantize_act_ex with a rotation or rule): DYNAMIC
+    global scale when g is None, else STATIC g.  ws: scratch of at least
+    fp4_workspace_bytes bytes; calls that may run concurrently (other
+    streams) need their own, else the shared per-device buffer is used."""
     _cuda_bf16_2d(x, "x")
     rows, K = x.shape
     dev = x.device
@@ -77,14 +80,22 @@ def quantize(x: torch.Tensor, fmt: int = NVFP4, layout: int = SCALES_MMA,
         ws = workspace(ws_bytes, dev)
     elif ws.numel() < ws_bytes:
         raise ValueError("workspace too small")
-    _check(L.fp4_quantize_act(x.data_ptr(), rows, K, fmt, layout, gmode, gt.data_ptr(),
-                              codes.data_ptr(), scales.data_ptr(), ws.data_ptr(), ws.numel(),
-                              _stream()), "fp4_quantize_act")
-    return Quantized(codes, scales, gt, fmt, layout, rows, K)
+    if hadamard or mx_rule:
+        _check(L.fp4_quantize_act_ex(x.data_ptr(), rows, K, fmt, layout, gmode,
+                                     L.opts(hadamard, mx_rule), gt.data_ptr(), codes.data_ptr(),
+                                     scales.data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
+               "fp4_quantize_act_ex")
+    else:
+        _check(L.fp4_quantize_act(x.data_ptr(), rows, K, fmt, layout, gmode, gt.data_ptr(),
+                                  codes.data_ptr(), scales.data_ptr(), ws.data_ptr(), ws.numel(),
+                                  _stream()), "fp4_quantize_act")
+    return Quantized(codes, scales, gt, fmt, layout, rows, K, hadamard, mx_rule)
 
 
-def quantize_weights(w: torch.Tensor, fmt: int = NVFP4) -> Quantized:
-    """fp4_quantize_weights: one-time, MMA scale layout, DYNAMIC g."""
+def quantize_weights(w: torch.Tensor, fmt: int = NVFP4, hadamard: int = 0,
+                     mx_rule: int = 0) -> Quantized:
+    """fp4_quantize_weights (fp4_quantize_weights_ex with a rotation or
+    rule): one-time, MMA scale layout, DYNAMIC g."""
     _cuda_bf16_2d(w, "w")
     N, K = w.shape
     dev = w.device
@@ -93,10 +104,16 @@ def quantize_weights(w: torch.Tensor, fmt: int = NVFP4) -> Quantized:
                          device=dev)
     g = torch.ones(1, dtype=torch.float32, device=dev)
     ws = workspace(L.fp4_workspace_bytes(N, 0, K, fmt), dev)
-    _check(L.fp4_quantize_weights(w.data_ptr(), N, K, fmt, codes.data_ptr(), scales.data_ptr(),
-                                  g.data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
-           "fp4_quantize_weights")
-    return Quantized(codes, scales, g, fmt, SCALES_MMA, N, K)
+    if hadamard or mx_rule:
+        _check(L.fp4_quantize_weights_ex(w.data_ptr(), N, K, fmt, L.opts(hadamard, mx_rule),
+                                         codes.data_ptr(), scales.data_ptr(), g.data_ptr(),
+                                         ws.data_ptr(), ws.numel(), _stream()),
+               "fp4_quantize_weights_ex")
+    else:
+        _check(L.fp4_quantize_weights(w.data_ptr(), N, K, fmt, codes.data_ptr(),
+                                      scales.data_ptr(), g.data_ptr(), ws.data_ptr(), ws.numel(),
+                                      _stream()), "fp4_quantize_weights")
+    return Quantized(codes, scales, g, fmt, SCALES_MMA, N, K, hadamard, mx_rule)
 
 
 def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
@@ -105,6 +122,8 @@ def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
     shape is chosen for (0 = all; concurrent GEMMs each take a share)."""
     if a.fmt != w.fmt or a.K != w.K or a.layout != SCALES_MMA or w.layout != SCALES_MMA:
         raise ValueError("operands must share format and K and use the MMA scale layout")
+    if a.hadamard != w.hadamard:
+        raise ValueError("a rotated activation needs weights rotated with the same order")
     M, N, K = a.rows, w.rows, a.K
     dev = a.codes.device
     if out is None:
@@ -113,6 +132,86 @@ def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
     _check(L.fp4_gemm(a.codes.data_ptr(), a.scales.data_ptr(), a.g.data_ptr(),
                       w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(), M, N, K, a.fmt,
                       out.data_ptr(), out.stride(0), o, None, 0, max_sms, _stream()), "fp4_gemm")
+    return out
+
+
+def gemm_quant(a: Quantized, w: Quantized, out_fmt: int = NVFP4, out_layout: int = SCALES_MMA,
+               g_out: torch.Tensor | None = None, hadamard: int = 0, mx_rule: int = 0,
+               with_c: bool = False, max_sms: int = 0):
+    """fp4_gemm_quant: C = alpha * A_hat . W_hat^T rounded to bf16 and
+    quantized in the GEMM's epilogue as the next layer's activation (NVFP4
+    with the STATIC global scale g_out, or MXFP4).  Returns (Quantized of
+    the [M, N] activation, bf16 C or None)."""
+    if a.fmt != w.fmt or a.K != w.K or a.layout != SCALES_MMA or w.layout != SCALES_MMA:
+        raise ValueError("operands must share format and K and use the MMA scale layout")
+    if a.hadamard != w.hadamard:
+        raise ValueError("a rotated activation needs weights rotated with the same order")
+    M, N, K = a.rows, w.rows, a.K
+    dev = a.codes.device
+    codes = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(max(L.fp4_scale_bytes(M, N, out_fmt, out_layout), 1), dtype=torch.uint8,
+                         device=dev)
+    if g_out is None:
+        g_out = torch.ones(1, dtype=torch.float32, device=dev)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if with_c else None
+    _check(L.fp4_gemm_quant(a.codes.data_ptr(), a.scales.data_ptr(), a.g.data_ptr(),
+                            w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(), M, N, K,
+                            a.fmt, out_fmt, out_layout, L.opts(hadamard, mx_rule),
+                            g_out.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                            c.data_ptr() if c is not None else None, N, None, 0, max_sms,
+                            _stream()), "fp4_gemm_quant")
+    return Quantized(codes, scales, g_out, out_fmt, out_layout, M, N, hadamard, mx_rule), c
+
+
+@dataclass
+class QuantizedExperts:
+    """E experts' weights [E, N, K] quantized one by one (MMA scale order),
+    stored back to back as fp4_gemm_grouped reads them."""
+    codes: torch.Tensor      # uint8 [E, N, K/2]
+    scales: torch.Tensor     # uint8 [E, per-expert scale bytes]
+    g: torch.Tensor          # float32 [E]
+    fmt: int
+    E: int
+    N: int
+    K: int
+
+
+def quantize_experts(w: torch.Tensor, fmt: int = NVFP4) -> QuantizedExperts:
+    """fp4_quantize_weights per expert of a bf16 [E, N, K] tensor (each with
+    its own DYNAMIC global scale), into one stacked buffer."""
+    if not w.is_cuda or w.dtype != torch.bfloat16 or w.dim() != 3 or not w.is_contiguous():
+        raise ValueError("w must be a contiguous 3-D bf16 CUDA tensor [E, N, K]")
+    E, N, K = w.shape
+    dev = w.device
+    sfb = L.fp4_scale_bytes(N, K, fmt, SCALES_MMA)
+    codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((E, sfb), dtype=torch.uint8, device=dev)
+    g = torch.ones(E, dtype=torch.float32, device=dev)
+    ws = workspace(L.fp4_workspace_bytes(N, 0, K, fmt), dev)
+    for e in range(E):
+        _check(L.fp4_quantize_weights(w[e].data_ptr(), N, K, fmt, codes[e].data_ptr(),
+                                      scales[e].data_ptr(), g[e:].data_ptr(), ws.data_ptr(),
+                                      ws.numel(), _stream()), "fp4_quantize_weights")
+    return QuantizedExperts(codes, scales, g, fmt, E, N, K)
+
+
+def gemm_grouped(a: Quantized, w: QuantizedExperts, offsets: torch.Tensor,
+                 out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                 max_sms: int = 0) -> torch.Tensor:
+    """fp4_gemm_grouped: rows [offsets[e], offsets[e+1]) of the quantized
+    activation times expert e's weights.  offsets: int32 CUDA tensor [E+1]."""
+    if a.fmt != w.fmt or a.K != w.K or a.layout != SCALES_MMA:
+        raise ValueError("operands must share format and K and use the MMA scale layout")
+    if (not offsets.is_cuda or offsets.dtype != torch.int32 or offsets.numel() != w.E + 1):
+        raise ValueError("offsets must be an int32 CUDA tensor of E + 1 entries")
+    M, N, K = a.rows, w.N, a.K
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.codes.device)
+    o = L.FP4_OUT_F32 if out.dtype == torch.float32 else L.FP4_OUT_BF16
+    _check(L.fp4_gemm_grouped(a.codes.data_ptr(), a.scales.data_ptr(), a.g.data_ptr(),
+                              w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(),
+                              offsets.data_ptr(), w.E, M, N, K, a.fmt, out.data_ptr(),
+                              out.stride(0), o, None, 0, max_sms, _stream()), "fp4_gemm_grouped")
     return out
 
 
@@ -127,10 +226,11 @@ def gemm_plan(M: int, N: int, K: int, fmt: int = NVFP4, max_sms: int = 0) -> tup
 def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
                g_a: torch.Tensor | None = None, out: torch.Tensor | None = None,
                g_out: torch.Tensor | None = None, ws: torch.Tensor | None = None,
-               max_sms: int = 0) -> torch.Tensor:
-    """fp4_gemm_fused: quantize x (M <= 32) on the fly and multiply with w.
-    ws: as for quantize (concurrent calls need their own); max_sms as for
-    gemm."""
+               max_sms: int = 0, mx_rule: int = 0) -> torch.Tensor:
+    """fp4_gemm_fused (fp4_gemm_fused_ex when w is rotated or a rule is
+    given): quantize x (M <= 32) on the fly and multiply with w; x is
+    rotated with w's order.  ws: as for quantize (concurrent calls need
+    their own); max_sms as for gemm."""
     _cuda_bf16_2d(x, "x")
     M, K = x.shape
     N = w.rows
@@ -146,10 +246,17 @@ def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
         ws = workspace(need, dev)
     elif ws.numel() < need:
         raise ValueError("workspace too small")
-    _check(L.fp4_gemm_fused(x.data_ptr(), w.codes.data_ptr(), w.scales.data_ptr(),
-                            w.g.data_ptr(), M, N, K, w.fmt, gmode, g_a.data_ptr(),
-                            out.data_ptr(), out.stride(0), o, ws.data_ptr(), ws.numel(),
-                            max_sms, _stream()), "fp4_gemm_fused")
+    if w.hadamard or mx_rule:
+        _check(L.fp4_gemm_fused_ex(x.data_ptr(), w.codes.data_ptr(), w.scales.data_ptr(),
+                                   w.g.data_ptr(), M, N, K, w.fmt, gmode,
+                                   L.opts(w.hadamard, mx_rule), g_a.data_ptr(), out.data_ptr(),
+                                   out.stride(0), o, ws.data_ptr(), ws.numel(), max_sms,
+                                   _stream()), "fp4_gemm_fused_ex")
+    else:
+        _check(L.fp4_gemm_fused(x.data_ptr(), w.codes.data_ptr(), w.scales.data_ptr(),
+                                w.g.data_ptr(), M, N, K, w.fmt, gmode, g_a.data_ptr(),
+                                out.data_ptr(), out.stride(0), o, ws.data_ptr(), ws.numel(),
+                                max_sms, _stream()), "fp4_gemm_fused")
     return out
 
 

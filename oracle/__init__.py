@@ -313,6 +313,20 @@ def gemm(a_hat: np.ndarray, w_hat: np.ndarray) -> np.ndarray:
     return np.asarray(a_hat, np.float64) @ np.asarray(w_hat, np.float64).T
 
 
+def gemm_grouped(a_hat: np.ndarray, w_hats, offsets) -> np.ndarray:
+    """Grouped GEMM by its plain definition: rows [offsets[e], offsets[e+1])
+    of A_hat times expert e's W_hat^T (binary64, the library matmul per
+    group); rows outside every group stay 0."""
+    a = np.asarray(a_hat, np.float64)
+    N = np.asarray(w_hats[0]).shape[0]
+    c = np.zeros((a.shape[0], N), np.float64)
+    for e, w in enumerate(w_hats):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            c[lo:hi] = a[lo:hi] @ np.asarray(w, np.float64).T
+    return c
+
+
 def w4a4_reference(a_bf16, w_bf16, fmt: int, g_a: float | None = None,
                    g_w: float | None = None):
     """Quantize both operands by the definition, then C = A_hat . W_hat^T.

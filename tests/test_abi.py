@@ -104,3 +104,19 @@ def test_no_gpu_means_no_device_status(lib):
     fake = ctypes.c_void_p(1 << 20)
     st = L.fp4_quantize_act(fake, 4, 256, 0, 0, 0, fake, fake, fake, fake, 1 << 16, None)
     assert st in (L.FP4_ERR_NO_DEVICE,)
+
+
+def test_quant_options_checked_before_any_launch(lib):
+    fake = ctypes.c_void_p(1 << 20)
+    qx = L.fp4_quantize_act_ex
+    assert qx(fake, 4, 256, 0, 0, 0, L.opts(8, 0), fake, fake, fake, fake, 1 << 16, None) == \
+        L.FP4_ERR_INVALID_ARG                                         # order 8
+    assert qx(fake, 4, 256, 0, 0, 0, L.opts(0, 1), fake, fake, fake, fake, 1 << 16, None) == \
+        L.FP4_ERR_INVALID_ARG                                         # OAS with NVFP4
+    assert qx(fake, 4, 100, 1, 0, 0, L.opts(32, 1), fake, fake, fake, fake, 1 << 16, None) == \
+        L.FP4_ERR_UNSUPPORTED_SHAPE                                   # K % 32
+    assert L.fp4_quantize_weights_ex(fake, 4, 256, 1, L.opts(16, 5), fake, fake, fake, fake,
+                                     1 << 16, None) == L.FP4_ERR_INVALID_ARG
+    fx = L.fp4_gemm_fused_ex
+    assert fx(fake, fake, fake, fake, 8, 16, 256, 0, 0, L.opts(64, 0), fake, fake, 16, 0, fake,
+              1 << 30, 0, None) == L.FP4_ERR_INVALID_ARG
