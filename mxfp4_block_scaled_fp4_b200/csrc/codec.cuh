@@ -135,42 +135,94 @@ __device__ __forceinline__ void unpack16(uint4 p, uint4 q, float f[16]) {
   }
 }
 
+// Two binary32 lanes in one 64-bit register and their packed arithmetic
+// (one IEEE rounding per lane, as the scalar operations).
+__device__ __forceinline__ unsigned long long f2(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long add_f2(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long sub_f2(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long mul_f2(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// RN(a * b + c) per lane; with b = +-1 it is RN(c +- a), one rounding.
+__device__ __forceinline__ unsigned long long fma_f2(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 // The in-unit stages h = 1, 2, 4, 8 of the transform, then (n = 16) the
 // scaling; n = 32 adds the cross-lane stage h = 16 (every lane of the warp
 // must take part) before it.  `odd` = this unit is the upper half of its
-// 32-value block.
+// 32-value block.  Stage h = 1 pairs the two lanes of a packed register
+// (scalar adds); from h = 2 on a pair of registers (i, i + h) moves as one
+// packed add and one packed subtract.
 template <int N>
 __device__ __forceinline__ void rotate_unit(float f[16], float scale, bool odd) {
 #pragma unroll
-  for (int h = 1; h < 16; h *= 2) {
+  for (int i = 0; i < 16; i += 2) {
+    const float a = f[i], b = f[i + 1];
+    f[i] = __fadd_rn(a, b);
+    f[i + 1] = __fsub_rn(a, b);
+  }
+  unsigned long long P[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if ((i & h) == 0) {
-        const float a = f[i], b = f[i + h];
-        f[i] = __fadd_rn(a, b);
-        f[i + h] = __fsub_rn(a, b);
+  for (int k = 0; k < 8; ++k) P[k] = f2(f[2 * k], f[2 * k + 1]);
+#pragma unroll
+  for (int hh = 1; hh < 8; hh *= 2) {        // h = 2 hh
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if ((k & hh) == 0) {
+        const unsigned long long a = P[k], b = P[k + hh];
+        P[k] = add_f2(a, b);
+        P[k + hh] = sub_f2(a, b);
       }
     }
   }
   if (N == 32) {
+    // lower half: own + other; upper half: other - own (= own * -1 + other)
+    const float sg = odd ? -1.0f : 1.0f;
+    const unsigned long long S = f2(sg, sg);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float o = __shfl_xor_sync(0xFFFFFFFFu, f[i], 1);
-      // lower half: own + other; upper half: lower (the other) - own
-      f[i] = odd ? __fsub_rn(o, f[i]) : __fadd_rn(f[i], o);
+    for (int k = 0; k < 8; ++k) {
+      float lo, hi;
+      f2_split(P[k], lo, hi);
+      const float olo = __shfl_xor_sync(0xFFFFFFFFu, lo, 1);
+      const float ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, 1);
+      P[k] = fma_f2(P[k], S, f2(olo, ohi));
     }
   }
+  const unsigned long long SC = f2(scale, scale);   // a power of two: exact
 #pragma unroll
-  for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(f[i], scale);   // exact: a power of two
+  for (int k = 0; k < 8; ++k) f2_split(mul_f2(P[k], SC), f[2 * k], f[2 * k + 1]);
 }
 
 // Largest magnitude of 16 floats as binary32 magnitude bits (Inf and NaN
 // order above every finite value).
 __device__ __forceinline__ unsigned mag_max16(const float f[16]) {
-  unsigned m = 0;
+  // max.NaN.xorsign.abs: the magnitude of the result is the larger of the
+  // two magnitudes (a NaN wins); the sign bit is dropped at the end
+  float m = f[0];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) m = max(m, __float_as_uint(f[i]) & 0x7FFFFFFFu);
-  return m;
+  for (int i = 1; i < 16; ++i) asm("max.NaN.xorsign.abs.f32 %0, %0, %1;" : "+f"(m) : "f"(f[i]));
+  return __float_as_uint(m) & 0x7FFFFFFFu;
 }
 
 // 8 floats times r -> 8 packed E2M1 codes (element i in nibble i); the
