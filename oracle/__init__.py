@@ -87,6 +87,10 @@ def _declare(L):
     L.orc_mxfp4_quantize_f32.argtypes = [P, i64, i64, ctypes.c_int, P, P]
     L.orc_hadamard_f32.restype = ctypes.c_int
     L.orc_hadamard_f32.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, P]
+    L.orc_mbs_sigma.restype = ctypes.c_float
+    L.orc_mbs_sigma.argtypes = [ctypes.c_float]
+    L.orc_mxfp4_mbs_quantize.restype = ctypes.c_int
+    L.orc_mxfp4_mbs_quantize.argtypes = [P, i64, i64, ctypes.c_int, P, P, P]
     L.orc_e2m1_encode_array.restype = None
     L.orc_e2m1_encode_array.argtypes = [P, i64, P]
     L.orc_e4m3_encode_array.restype = None
@@ -279,6 +283,26 @@ def quantize_ex(x, fmt: int, g: float | None = None, hadamard_n: int = 0,
     else:
         return quantize(x, fmt, g)
     return quantize_f32(xf, fmt, g, rule)
+
+
+def mbs_sigma(amax_row: float) -> float:
+    """R9: the macro scale of a row whose largest magnitude is amax_row."""
+    return float(lib().orc_mbs_sigma(amax_row))
+
+
+def quantize_mxfp4_mbs(x, rule: int = OCP):
+    """R9: MXFP4 with one binary32 macro scale per row.  Returns (codes,
+    row-major E8M0 scales, sigma [rows] float32)."""
+    x = _as_bf16_bits(x)
+    rows, K = x.shape
+    codes = np.empty((rows, K // 2), np.uint8)
+    scales = np.empty((rows, K // 32), np.uint8)
+    sigma = np.empty(rows, np.float32)
+    rc = lib().orc_mxfp4_mbs_quantize(_ptr(x), rows, K, int(rule), _ptr(sigma), _ptr(codes),
+                                      _ptr(scales))
+    if rc != 0:
+        raise ValueError(f"bad shape or rule: {x.shape}, rule {rule}")
+    return codes, scales, sigma
 
 
 def dequant(codes: np.ndarray, scales: np.ndarray, fmt: int, g: float = 1.0):

@@ -55,6 +55,17 @@
  *     with b <= 6 * 2^e, i.e. e = floor(log2 b) - 2 when b / 2^floor(log2 b)
  *     <= 1.5 and one more otherwise, clamped to [-127, 127] (-127 for a zero
  *     block).  R5 is the OCP rule, which lets values in (6, 8) * 2^e clip.
+ *  R9 MXFP4 macro-block scaling (MBS; [DIA], same section: a second-level
+ *     scale over a "macro-block" grouping several 32-blocks, the base
+ *     format unchanged, bringing MXFP4 close to two-level scaling): the
+ *     macro-block is one row (all K / 32 blocks of a token or an output
+ *     channel, so that the GEMM applies the second level in its epilogue
+ *     as sigma_a[m] * sigma_w[n]).  Per row: A = max |x| (exact);
+ *     t = RN(A / 6); sigma = t * 2^-floor(log2 t) (exact: t's significand,
+ *     in [1, 2)); sigma = 1 when A == 0; rho = RN(1 / sigma);
+ *     x' = RN(x * rho); then the MXFP4 block quantizer (R5 or R8) on x'.
+ *     The row's largest block then sits at the top of its E2M1 range;
+ *     x_hat = sigma * 2^e * q.
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC
  * (oracle/build.py).  FP32 arithmetic is SSE binary32 on x86-64
@@ -362,6 +373,48 @@ int orc_mxfp4_quantize(const uint16_t* x, long rows, long K,
             for (int i = 0; i < 32; ++i)
                 xf[i] = orc_bf16_to_f32(x[r * K + b * 32 + i]);
             scales[r * nb + b] = (uint8_t)mxfp4_block(xf, 0, q);
+            for (int j = 0; j < 16; ++j)
+                codes[r * (K / 2) + b * 16 + j] =
+                    (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------ macro-block scaling (R9) -- */
+
+/* The macro scale of a row from its largest magnitude A (R9). */
+float orc_mbs_sigma(float A)
+{
+    if (A == 0.0f) return 1.0f;
+    float t = A / 6.0f;
+    int ex = floor_log2_f32(t);
+    return (float)ldexp((double)t, -ex);       /* exact: t's significand */
+}
+
+/* MXFP4 with a macro scale per row (R9): sigma[rows] out, codes
+ * [rows, K/2], scales [rows, K/32] (rule as in orc_mxfp4_quantize_f32). */
+int orc_mxfp4_mbs_quantize(const uint16_t* x, long rows, long K, int rule,
+                           float* sigma, uint8_t* codes, uint8_t* scales)
+{
+    if (rows < 0 || K <= 0 || K % 32 != 0 || rule < 0 || rule > 1) return ORC_BAD_SHAPE;
+    const long nb = K / 32;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        float A = 0.0f;
+        for (long k = 0; k < K; ++k) {
+            float a = fabsf(orc_bf16_to_f32(x[r * K + k]));
+            if (a > A) A = a;
+        }
+        const float sg = orc_mbs_sigma(A);
+        const float rho = 1.0f / sg;
+        sigma[r] = sg;
+        for (long b = 0; b < nb; ++b) {
+            float xf[32];
+            unsigned char q[32];
+            for (int i = 0; i < 32; ++i)
+                xf[i] = orc_bf16_to_f32(x[r * K + b * 32 + i]) * rho;
+            scales[r * nb + b] = (uint8_t)mxfp4_block(xf, rule, q);
             for (int j = 0; j < 16; ++j)
                 codes[r * (K / 2) + b * 16 + j] =
                     (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
