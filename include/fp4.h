@@ -138,6 +138,20 @@ typedef enum { FP4_MX_RULE_OCP = 0, FP4_MX_RULE_OAS = 1 } fp4_mx_rule_t;
 typedef struct {
     int hadamard;
     fp4_mx_rule_t mx_rule;
+    /* MXFP4 macro-block scaling (MBS; "FP4 n'existe pas", section "L'ecart
+     * de qualite -- et comment il se reduit": a second-level scale over a
+     * macro-block of several 32-blocks, the base format unchanged).  Here a
+     * macro-block is one row (all K / 32 blocks of a token or an output
+     * channel), so that fp4_gemm_mbs applies the second level in its
+     * epilogue.  NULL: off.  Otherwise a DEVICE array of `rows` floats that
+     * the call writes: per row, with A its largest magnitude, sigma = the
+     * significand of RN(A / 6) (in [1, 2); 1 for an all-zero row); the row
+     * is multiplied by RN(1 / sigma) (one rounding per value) before the
+     * MXFP4 quantizer (mx_rule applies), so that x_hat = sigma * 2^e * q.
+     * MXFP4 only, without rotation (FP4_ERR_INVALID_ARG otherwise); not
+     * accepted by fp4_gemm_fused_ex or fp4_gemm_quant.  A non-finite row
+     * maximum is reported as FP4_ERR_NONFINITE by fp4_device_status. */
+    float* mbs_scale;
 } fp4_quant_opts_t;
 
 /* fp4_quantize_act with options (above).  opts == NULL is fp4_quantize_act.
@@ -254,6 +268,21 @@ fp4_status_t fp4_gemm_quant(const uint8_t* a_codes, const uint8_t* a_scales, con
                             const float* g_out, uint8_t* out_codes, uint8_t* out_scales,
                             void* C, int ldc, void* ws, size_t ws_bytes, int max_sms,
                             void* stream);
+
+/* MXFP4 GEMM with macro-block scaling: A and W quantized with
+ * fp4_quant_opts_t.mbs_scale (fp4_quantize_act_ex, fp4_quantize_weights_ex)
+ * and their per-row macro scales sigma_a [M], sigma_w [N] (device arrays):
+ *     C[m, n] = RN(RN(sigma_a[m] * sigma_w[n]) * acc[m, n]),
+ * acc the FP32 block-scaled accumulation of the MXFP4 codes and E8M0
+ * scales (as fp4_gemm), bf16 or fp32 out.  The launch shape is fp4_gemm's
+ * without a K split.  Shapes, alignment and errors as fp4_gemm (sigma
+ * pointers 4-byte aligned, never NULL).  "FP4 n'existe pas", section
+ * "L'ecart de qualite -- et comment il se reduit" (the GEMM pays a small
+ * overhead for the second level). */
+fp4_status_t fp4_gemm_mbs(const uint8_t* a_codes, const uint8_t* a_scales, const float* sigma_a,
+                          const uint8_t* w_codes, const uint8_t* w_scales, const float* sigma_w,
+                          int M, int N, int K, void* C, int ldc, fp4_out_t out,
+                          void* ws, size_t ws_bytes, int max_sms, void* stream);
 
 /* Grouped block-scaled FP4 GEMM (mixture of experts: many per-expert GEMMs
  * in one launch).  Group e (0 <= e < E) is rows [offsets[e], offsets[e+1])

@@ -36,7 +36,7 @@ def _stale(target, deps):
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
     os.makedirs(OBJ_DIR, exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     hdrs = [d for d in _deps() if not d.endswith(".cu")]
     for src in sources():
         obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
@@ -47,7 +47,13 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
                 cmd.insert(1, "-Xptxas=-v")
             if verbose:
                 print(" ".join(cmd))
-            subprocess.run(cmd, check=True)
+            cmds.append(cmd)
+    # the translation units compile independently: run them side by side
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
+        for r in list(ex.map(lambda c: subprocess.run(c), cmds)):
+            if r.returncode != 0:
+                raise subprocess.CalledProcessError(r.returncode, r.args)
     if force or _stale(LIB, objs):
         tmp = LIB + f".tmp{os.getpid()}"
         cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lrt",

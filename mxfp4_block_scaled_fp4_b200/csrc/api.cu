@@ -91,6 +91,7 @@ struct Opts {
   int rot = 0;
   float rot_scale = 1.0f;
   int rule = 0;
+  float* mbs = nullptr;
 };
 fp4_status_t parse_opts(const fp4_quant_opts_t* o, fp4_format_t fmt, bool weights, Opts* out) {
   *out = Opts{};
@@ -98,6 +99,11 @@ fp4_status_t parse_opts(const fp4_quant_opts_t* o, fp4_format_t fmt, bool weight
   if (o->hadamard != 0 && o->hadamard != 16 && o->hadamard != 32) return FP4_ERR_INVALID_ARG;
   if (o->mx_rule != FP4_MX_RULE_OCP && o->mx_rule != FP4_MX_RULE_OAS) return FP4_ERR_INVALID_ARG;
   if (fmt == FP4_NVFP4 && o->mx_rule != FP4_MX_RULE_OCP) return FP4_ERR_INVALID_ARG;
+  if (o->mbs_scale) {
+    if (fmt != FP4_MXFP4 || o->hadamard != 0) return FP4_ERR_INVALID_ARG;
+    if (!aligned4(o->mbs_scale)) return FP4_ERR_MISALIGNED;
+    out->mbs = o->mbs_scale;
+  }
   out->rot = o->hadamard;
   out->rule = o->mx_rule == FP4_MX_RULE_OAS ? 1 : 0;
   if (o->hadamard) {
@@ -143,6 +149,7 @@ fp4_status_t quantize_common(const void* x, int rows, int K, fp4_format_t fmt,
   a.rot = op.rot;
   a.rot_scale = op.rot_scale;
   a.rule = op.rule;
+  a.mbs_sigma = op.mbs;
   // The amax pass (DYNAMIC) and the quantize pass, each a programmatic
   // dependent of the kernel before it (each waits for its predecessor before
   // reading), so its launch overlaps the predecessor's tail.  No pass
@@ -262,6 +269,7 @@ fp4_status_t fp4_gemm_quant(const uint8_t* a_codes, const uint8_t* a_scales, con
   if (out_layout != FP4_SCALES_MMA && out_layout != FP4_SCALES_ROWMAJOR) return FP4_ERR_INVALID_ARG;
   Opts op;
   if ((st = parse_opts(out_opts, out_fmt, false, &op)) != FP4_OK) return st;
+  if (op.mbs) return FP4_ERR_INVALID_ARG;   // no macro-block scaling in the emitting epilogue
   if (max_sms < 0) return FP4_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (N % 32 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;   // N is the next layer's K
@@ -302,6 +310,45 @@ fp4_status_t fp4_gemm_quant(const uint8_t* a_codes, const uint8_t* a_scales, con
   a.qo.rot_scale = op.rot_scale;
   a.qo.nsf = fp4::nsf_of(N, a.qo.fmt);
   a.qo.ncb = fp4::ncb_of(a.qo.nsf);
+  return from_cuda(fp4::launch_gemm(a, static_cast<cudaStream_t>(stream)));
+}
+
+fp4_status_t fp4_gemm_mbs(const uint8_t* a_codes, const uint8_t* a_scales, const float* sigma_a,
+                          const uint8_t* w_codes, const uint8_t* w_scales, const float* sigma_w,
+                          int M, int N, int K, void* C, int ldc, fp4_out_t out, void* ws,
+                          size_t ws_bytes, int max_sms, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  fp4_status_t st;
+  if (out != FP4_OUT_BF16 && out != FP4_OUT_F32) return FP4_ERR_INVALID_ARG;
+  if (max_sms < 0) return FP4_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || (st = check_rows_k(M, K)) != FP4_OK) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return FP4_OK;
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !C || !sigma_a || !sigma_w)
+    return FP4_ERR_INVALID_ARG;
+  if (ldc < N) return FP4_ERR_INVALID_ARG;
+  const int esize = out == FP4_OUT_F32 ? 4 : 2;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(C) || (static_cast<long long>(ldc) * esize) % 16 != 0 || !aligned4(sigma_a) ||
+      !aligned4(sigma_w))
+    return FP4_ERR_MISALIGNED;
+  if ((st = device_ok()) != FP4_OK) return st;
+  fp4::GemmArgs a{};
+  a.a_codes = a_codes;
+  a.a_scales = a_scales;
+  a.w_codes = w_codes;
+  a.w_scales = w_scales;
+  a.sigma_a = sigma_a;
+  a.sigma_w = sigma_w;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.fmt = FP4_MXFP4;
+  a.C = C;
+  a.ldc = ldc;
+  a.out_mode = out == FP4_OUT_F32 ? 5 : 4;
+  a.max_sms = max_sms;
   return from_cuda(fp4::launch_gemm(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -379,6 +426,7 @@ fp4_status_t fp4_gemm_fused_ex(const void* x, const uint8_t* w_codes, const uint
   if ((st = check_format(fmt)) != FP4_OK) return st;
   Opts op;
   if ((st = parse_opts(opts, fmt, false, &op)) != FP4_OK) return st;
+  if (op.mbs) return FP4_ERR_INVALID_ARG;   // the fused path has no macro-block scaling
   if (out != FP4_OUT_BF16 && out != FP4_OUT_F32) return FP4_ERR_INVALID_ARG;
   if (gmode != FP4_GLOBAL_DYNAMIC && gmode != FP4_GLOBAL_STATIC) return FP4_ERR_INVALID_ARG;
   if (max_sms < 0) return FP4_ERR_INVALID_ARG;

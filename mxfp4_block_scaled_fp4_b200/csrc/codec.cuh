@@ -286,4 +286,19 @@ __device__ __forceinline__ unsigned mxfp4_scale_f32(unsigned b_bits, int rule, f
   return static_cast<unsigned>(e + 127);
 }
 
+// MXFP4 macro-block scaling (the second-level scale of "FP4 n'existe pas",
+// section "L'ecart de qualite -- et comment il se reduit", read as one
+// binary32 scale per row): sigma = the significand of RN(A / 6) for the
+// row's largest magnitude A (in [1, 2); 1 when A == 0), exact from the bits.
+__device__ __forceinline__ float mbs_sigma(float A) {
+  if (A == 0.0f) return 1.0f;
+  const unsigned b = __float_as_uint(__fdiv_rn(A, 6.0f));
+  unsigned man = b & 0x7FFFFFu;
+  if (((b >> 23) & 0xFFu) == 0) {   // subnormal: normalise the significand
+    const int msb = 31 - __clz(man);
+    man = (man << (23 - msb)) & 0x7FFFFFu;
+  }
+  return __uint_as_float(0x3F800000u | man);
+}
+
 }  // namespace fp4

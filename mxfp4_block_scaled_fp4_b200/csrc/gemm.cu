@@ -80,7 +80,8 @@ struct Tile {
   static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128) ? (G ? 5 : 6) : 7;
   static constexpr int RING = STAGES * STAGE_BYTES;
   static constexpr int GTAB = G ? 4 * (2 * kMaxGroups + 2) : 0;   // group table (ints)
-  static constexpr int SMEM = RING + 1024 + 512 + GTAB;   // ring + alignment + barriers
+  static constexpr int SMEM = RING + 1024 + 512 + GTAB + 512;   // ring, alignment, barriers,
+                                                                // groups, reciprocals
   // tensor-memory columns between the B scales of consecutive atoms, and
   // per stage (A scales in the first 16)
   static constexpr int SFB_ATOM_COLS = 4 * SF_BLOCKS;
@@ -113,7 +114,9 @@ struct Params {
   int E;
   long long w_sf_bytes;
   int a_rowblocks;        // ceil(M / 128)
-  QuantOut qo;            // OUT >= 2: the emitted FP4 activation (C optional)
+  QuantOut qo;            // OUT 2, 3: the emitted FP4 activation (C optional)
+  const float* sigma_a;   // OUT 4, 5: macro-block scales of A rows [M] and W rows [N]
+  const float* sigma_w;
 };
 
 // Split-K: CTA d of a tile's cluster reduces accumulator rows
@@ -180,7 +183,8 @@ __device__ __forceinline__ void store8(void* C, long long off, float alpha, cons
 
 // OUT: 0 = bf16 C, 1 = fp32 C, 2 / 3 = C quantized to NVFP4 / MXFP4
 // (out_quant.cuh; no K split), with the bf16 C stored as well when p.C is
-// not null.
+// not null; 4 / 5 = bf16 / fp32 C scaled by sigma_a[m] sigma_w[n] (MXFP4
+// macro-block scaling; no K split) instead of alpha.
 template <int FMT, int OUT, int BN, int G = 0>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
@@ -207,6 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* gtab = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + 512);   // G = 1
+  float* r_tab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 512 + T::GTAB);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -310,8 +315,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   float alpha = 1.0f;
   if (FMT == 0 && warp >= 2 && warp < 6 && !G) alpha = __fmul_rn(*p.g_a, *p.g_w);
+  constexpr bool F32 = OUT == 1 || OUT == 5;       // fp32 C
+  constexpr bool QOUT = OUT == 2 || OUT == 3;      // FP4 activation out
+  constexpr bool MBS = OUT >= 4;                   // per-row x per-column scales
   QuantOutG qg{};
-  if (OUT >= 2 && warp >= 2 && warp < 6) qg = quant_out_g(p.qo);
+  if (QOUT && warp >= 2 && warp < 6) {
+    qg = quant_out_g(p.qo, r_tab, threadIdx.x - 64);
+    asm volatile("bar.sync 1, 128;" ::: "memory");   // the 4 epilogue warps
+  }
   bool acc_ok = false;   // split-K epilogue: this CTA's accumulator is complete
 
   constexpr int kAtomsPerStage = (FMT == 0) ? 4 : 2;   // scale atoms per 256 K
@@ -580,7 +591,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const bool row_ok = row < row_end;
         const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL;
-        if (OUT != 1) {
+        const float arow = MBS ? __ldg(p.sigma_a + min(row, p.M - 1)) : alpha;
+        if (!F32) {
           // bf16: the whole row fits in registers once packed, so the
           // accumulator is released before any global store is issued
           uint32_t packed[BN / 2];
@@ -591,8 +603,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const float lo = __fmul_rn(alpha, __uint_as_float(r[2 * j]));
-              const float hi = __fmul_rn(alpha, __uint_as_float(r[2 * j + 1]));
+              const int n = nt * BN + 32 * c + 2 * j;
+              const float lo =
+                  __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n, p.N), __uint_as_float(r[2 * j]));
+              const float hi =
+                  __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 1, p.N), __uint_as_float(r[2 * j + 1]));
               __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
               packed[16 * c + j] = *reinterpret_cast<uint32_t*>(&h);
             }
@@ -600,11 +615,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(acc_empty);
-          if (OUT >= 2) {
+          if (QOUT) {
             const bool pad = p.qo.layout == 0 && !row_ok && row < (p.M + 127) / 128 * 128;
-            quant_out_row<BN, OUT - 2>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N);
+            quant_out_row<BN, QOUT ? OUT - 2 : 0>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N);
           }
-          if (row_ok && (OUT == 0 || p.C != nullptr)) {
+          if (row_ok && (!QOUT || p.C != nullptr)) {
             uint16_t* out = static_cast<uint16_t*>(p.C) + static_cast<long long>(row) * p.ldc;
 #pragma unroll
             for (int v = 0; v < BN / 8; ++v) {
@@ -631,11 +646,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
               if (n0 + 4 * v < p.N) {
+                const int n = n0 + 4 * v;
                 float4 o;
-                o.x = __fmul_rn(alpha, __uint_as_float(r[4 * v + 0]));
-                o.y = __fmul_rn(alpha, __uint_as_float(r[4 * v + 1]));
-                o.z = __fmul_rn(alpha, __uint_as_float(r[4 * v + 2]));
-                o.w = __fmul_rn(alpha, __uint_as_float(r[4 * v + 3]));
+                o.x = __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n, p.N), __uint_as_float(r[4 * v + 0]));
+                o.y = __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 1, p.N), __uint_as_float(r[4 * v + 1]));
+                o.z = __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 2, p.N), __uint_as_float(r[4 * v + 2]));
+                o.w = __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 3, p.N), __uint_as_float(r[4 * v + 3]));
                 *reinterpret_cast<float4*>(out + 4 * v) = o;
               }
             }
@@ -723,7 +739,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] = (src == 0) ? x[i] : __fadd_rn(acc[i], x[i]);
           }
-          store8<OUT == 1>(p.C, (static_cast<long long>(mt) * BM + lo + lr) * p.ldc + nt * BN + 8 * g,
+          store8<F32>(p.C, (static_cast<long long>(mt) * BM + lo + lr) * p.ldc + nt * BN + 8 * g,
                           alpha, acc);
         }
       }
@@ -889,6 +905,11 @@ cudaError_t launch_bn(const GemmArgs& a, Params p, int splits, cudaStream_t s) {
   static const L table[2][4] = {
       {launch_typed<0, 0, BN>, launch_typed<0, 1, BN>, launch_typed<0, 2, BN>, launch_typed<0, 3, BN>},
       {launch_typed<1, 0, BN>, launch_typed<1, 1, BN>, launch_typed<1, 2, BN>, launch_typed<1, 3, BN>}};
+  if (a.out_mode >= 4) {   // macro-block scaling: MXFP4 only
+    if (a.fmt != 1) return cudaErrorInvalidValue;
+    return a.out_mode == 5 ? launch_typed<1, 5, BN>(ma, mw, p, grid, s)
+                           : launch_typed<1, 4, BN>(ma, mw, p, grid, s);
+  }
   return table[a.fmt != 0][a.out_mode](ma, mw, p, grid, s);
 }
 
@@ -919,7 +940,9 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   p.watchdog = watchdog_ptr();
   if (!p.watchdog) return cudaErrorInvalidSymbol;
   p.qo = a.qo;
-  // the FP4-emitting epilogue quantizes whole rows of a tile: no K split
+  p.sigma_a = a.sigma_a;
+  p.sigma_w = a.sigma_w;
+  // the FP4-emitting and the macro-block-scaled epilogues take no K split
   const Shape sh = choose_shape(p.m_tiles, a.N, p.k_steps, sms, max_clusters_bn, a.out_mode < 2);
   if (sh.bn == 64) return launch_bn<64>(a, p, sh.splits, s);
   if (sh.bn == 128) return launch_bn<128>(a, p, sh.splits, s);

@@ -71,7 +71,8 @@ constexpr int RING_BYTES = STAGES * (A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE);
 // (4 KiB each, 128-byte swizzle) that TMA stores drain to C
 constexpr int OUT_BUF = 32 * 128;
 constexpr int OUT_BYTES = 4 * 2 * OUT_BUF;
-constexpr int SMEM_BYTES = RING_BYTES + OUT_BYTES + 1024 + 256;
+constexpr int RTAB_BYTES = 512;          // FP4-emitting epilogue: 128 reciprocals
+constexpr int SMEM_BYTES = RING_BYTES + OUT_BYTES + RTAB_BYTES + 1024 + 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = 256;
@@ -96,7 +97,9 @@ struct Params {
   int a_rowblocks;        // ceil(M / 128)
   int w_rowblocks;        // ceil(N / 128)
   unsigned* watchdog;
-  QuantOut qo;            // OUT >= 2: the emitted FP4 activation (C optional)
+  QuantOut qo;            // OUT 2, 3: the emitted FP4 activation (C optional)
+  const float* sigma_a;   // OUT 4, 5: macro-block scales of A rows [M] and W rows [N]
+  const float* sigma_w;
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int& nt) {
@@ -110,7 +113,9 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int
 }
 
 // OUT: 0 = bf16 C, 1 = fp32 C, 2 / 3 = C quantized to NVFP4 / MXFP4
-// (out_quant.cuh), with the bf16 C stored as well when p.C is not null.
+// (out_quant.cuh), with the bf16 C stored as well when p.C is not null;
+// 4 / 5 = bf16 / fp32 C scaled by sigma_a[m] sigma_w[n] (MXFP4 macro-block
+// scaling) instead of alpha.
 template <int FMT, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
@@ -126,7 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sSFA = sB + STAGES * B_STAGE;
   uint8_t* sSFB = sSFA + STAGES * SFA_STAGE;
   uint8_t* sOut = sSFB + STAGES * SFB_STAGE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_BYTES);
+  float* r_tab = reinterpret_cast<float*>(sOut + OUT_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_BYTES + RTAB_BYTES);
   uint64_t* sf_loaded = full + STAGES;
   uint64_t* empty = sf_loaded + STAGES;
   uint64_t* ready = empty + STAGES;
@@ -155,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_w);
-    if (OUT <= 1 || p.C != nullptr) prefetch_tensormap(&tm_c);
+    if (!(OUT == 2 || OUT == 3) || p.C != nullptr) prefetch_tensormap(&tm_c);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -396,7 +402,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
     uint8_t* sOutW = sOut + (warp - 2) * 2 * OUT_BUF;
     QuantOutG qg{};
-    if (OUT >= 2) qg = quant_out_g(p.qo);
+    constexpr bool F32 = OUT == 1 || OUT == 5;       // fp32 C
+    constexpr bool QOUT = OUT == 2 || OUT == 3;      // FP4 activation out
+    constexpr bool MBS = OUT >= 4;                   // per-row x per-column scales
+    if (QOUT) {
+      qg = quant_out_g(p.qo, r_tab, threadIdx.x - 64);
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // the 4 epilogue warps
+    }
     int it = 0;
     for (int t = first; t < n_tiles_total; t += stride, ++it) {
       int mt, nt;
@@ -410,7 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = mt * BM + static_cast<int>(rank) * HALF + quarter * 32 + lane;
       const bool row_ok = row < p.M;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL;
-      if (OUT != 1) {
+      // MBS: the row's scale (the column's comes with each value)
+      const float arow = MBS ? __ldg(p.sigma_a + min(row, p.M - 1)) : alpha;
+      if (!F32) {
         uint32_t packed[BN / 2];
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
@@ -419,8 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float lo = __fmul_rn(alpha, __uint_as_float(r[2 * j]));
-            const float hi = __fmul_rn(alpha, __uint_as_float(r[2 * j + 1]));
+            const int n = nt * BN + 32 * c + 2 * j;
+            const float lo = __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n, p.N), __uint_as_float(r[2 * j]));
+            const float hi =
+                __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 1, p.N), __uint_as_float(r[2 * j + 1]));
             __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
             packed[16 * c + j] = *reinterpret_cast<uint32_t*>(&h);
           }
@@ -437,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // buffers and 64-column TMA stores (rows past M and columns past N
         // are clipped by the store)
         const int row0 = mt * BM + static_cast<int>(rank) * HALF + quarter * 32;
-        if (row0 < p.M && (OUT == 0 || p.C != nullptr)) {
+        if (row0 < p.M && (!QOUT || p.C != nullptr)) {
 #pragma unroll
           for (int c = 0; c < BN / 64; ++c) {
             const int n0 = nt * BN + 64 * c;
@@ -461,9 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (OUT >= 2) {
+        if (QOUT) {
           const bool pad = p.qo.layout == 0 && !row_ok && row < p.a_rowblocks * HALF;
-          quant_out_row<BN, OUT - 2>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N);
+          quant_out_row<BN, QOUT ? OUT - 2 : 0>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N);
         }
       } else {
         // fp32: 32-column chunks leave through the warp's two swizzled
@@ -496,12 +512,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           const uint32_t rowaddr = smem_u32(buf) + lane * 128;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
+          for (int j = 0; j < 8; ++j) {
+            const int n = n0 + 4 * j;
             sts128(rowaddr + ((j ^ (lane & 7)) << 4),
-                   __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[4 * j + 0]))),
-                   __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[4 * j + 1]))),
-                   __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[4 * j + 2]))),
-                   __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[4 * j + 3]))));
+                   __float_as_uint(__fmul_rn(col_scale<MBS>(arow, p.sigma_w, n, p.N), __uint_as_float(r[4 * j + 0]))),
+                   __float_as_uint(__fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 1, p.N), __uint_as_float(r[4 * j + 1]))),
+                   __float_as_uint(__fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 2, p.N), __uint_as_float(r[4 * j + 2]))),
+                   __float_as_uint(__fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 3, p.N), __uint_as_float(r[4 * j + 3]))));
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -573,10 +591,11 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
   CUtensorMap ma, mw, mc;
   if (!make_code_map(&ma, a.a_codes, a.M, a.K, HALF)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, a.w_codes, a.N, a.K, HALF)) return cudaErrorInvalidValue;
-  if (a.out_mode >= 2 && !a.C)
+  const bool f32 = a.out_mode == 1 || a.out_mode == 5;
+  if ((a.out_mode == 2 || a.out_mode == 3) && !a.C)
     mc = ma;   // unused: no bf16 C beside the FP4 output
-  else if (a.out_mode == 1 ? !make_f32_out_map(&mc, a.C, a.M, a.N, a.ldc, 32)
-                           : !make_bf16_out_map(&mc, a.C, a.M, a.N, a.ldc, 32))
+  else if (f32 ? !make_f32_out_map(&mc, a.C, a.M, a.N, a.ldc, 32)
+               : !make_bf16_out_map(&mc, a.C, a.M, a.N, a.ldc, 32))
     return cudaErrorInvalidValue;
   Params p;
   p.a_scales = a.a_scales;
@@ -597,12 +616,19 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
   p.watchdog = watchdog_ptr();
   if (!p.watchdog) return cudaErrorInvalidSymbol;
   p.qo = a.qo;
+  p.sigma_a = a.sigma_a;
+  p.sigma_w = a.sigma_w;
   const int tiles = p.m_tiles * p.n_tiles;
   using L = cudaError_t (*)(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                             const Params&, int, int, cudaStream_t);
   static const L table[2][4] = {
       {launch_typed<0, 0>, launch_typed<0, 1>, launch_typed<0, 2>, launch_typed<0, 3>},
       {launch_typed<1, 0>, launch_typed<1, 1>, launch_typed<1, 2>, launch_typed<1, 3>}};
+  if (a.out_mode >= 4) {   // macro-block scaling: MXFP4 only
+    if (a.fmt != 1) return cudaErrorInvalidValue;
+    return a.out_mode == 5 ? launch_typed<1, 5>(ma, mw, mc, p, tiles, a.max_sms, s)
+                           : launch_typed<1, 4>(ma, mw, mc, p, tiles, a.max_sms, s);
+  }
   return table[a.fmt != 0][a.out_mode](ma, mw, mc, p, tiles, a.max_sms, s);
 }
 

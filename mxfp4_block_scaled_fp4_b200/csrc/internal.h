@@ -72,6 +72,9 @@ struct QuantArgs {
   float rot_scale = 1.0f;
   // MXFP4 scale rule: 0 = OCP (floor(log2 amax) - 2), 1 = overflow-aware.
   int rule = 0;
+  // MXFP4 macro-block scaling: one binary32 scale per row, written by the
+  // row pass and read by the quantize pass (rot must be 0)
+  float* mbs_sigma = nullptr;
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s, bool pdl = false);
 
@@ -97,6 +100,9 @@ namespace fp4 {
 struct GemmArgs {
   const uint8_t* a_codes; const uint8_t* a_scales; const float* g_a;
   const uint8_t* w_codes; const uint8_t* w_scales; const float* g_w;
+  // MXFP4 macro-block scaling: per-row scales of A [M] and W [N] (both
+  // null otherwise); C = sigma_a[m] * sigma_w[n] * acc
+  const float* sigma_a = nullptr; const float* sigma_w = nullptr;
   int M, N, K, fmt;
   void* C; int ldc;
   int out_mode;         // 0 bf16 C, 1 fp32 C, 2 / 3 NVFP4 / MXFP4 activation (+ bf16 C if C)

@@ -26,17 +26,25 @@ struct QuantOut {
   int nsf, ncb;         // scale columns of a row (N / B) and their 4-column groups
 };
 
-// Per-thread constants of the NVFP4 scale step from the STATIC g.
+// Per-thread constants of the NVFP4 scale step from the STATIC g, and the
+// reciprocals r = RN(1 / RN(s g)) of every scale byte s <= 0x7F in shared
+// memory (r_tab, 128 floats, filled by the 128 epilogue threads: it
+// depends on the scale byte alone, so no block computes a reciprocal).
 struct QuantOutG {
   float g, six_g, y6;
   bool fast_b;
+  const float* r_tab;
 };
-__device__ __forceinline__ QuantOutG quant_out_g(const QuantOut& q) {
+// Every epilogue thread calls this once (tid = 0..127); the caller
+// synchronizes the 128 threads before the first quant_out_row.
+__device__ __forceinline__ QuantOutG quant_out_g(const QuantOut& q, float* r_tab, int tid) {
   QuantOutG c;
   c.g = q.fmt == 0 ? *q.g : 1.0f;
   c.six_g = __fmul_rn(6.0f, c.g);
   c.y6 = __frcp_rn(c.six_g);
   c.fast_b = c.six_g >= 0x1p-40f && c.six_g <= 0x1p40f;
+  if (q.fmt == 0) r_tab[tid] = nvfp4_recip(static_cast<unsigned>(tid), c.g);
+  c.r_tab = r_tab;
   return c;
 }
 
@@ -45,6 +53,15 @@ __device__ __forceinline__ long long out_scale_offset(const QuantOut& q, long lo
   const long long atom = (r >> 7) * q.ncb + (c >> 2);
   const int rr = static_cast<int>(r & 127);
   return atom * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (c & 3);
+}
+
+// The epilogue's multiplier of accumulator column n: alpha, or with MXFP4
+// macro-block scaling (MBS) RN(sigma_a[row] * sigma_w[n]) -- `a` is then
+// sigma_a[row]; columns past N get 0 (never stored).
+template <bool MBS>
+__device__ __forceinline__ float col_scale(float a, const float* sigma_w, int n, int N) {
+  if (!MBS) return a;
+  return __fmul_rn(a, n < N ? __ldg(sigma_w + n) : 0.0f);
 }
 
 // In-thread rotation of a 32-value block held as two 16-value halves.
@@ -87,7 +104,7 @@ __device__ __forceinline__ void quant_out_row(const QuantOut& q, const QuantOutG
         if (FMT == 0) {
           s0 = nvfp4_scale_byte(m0, gc.six_g, gc.y6, gc.fast_b);
           s1 = nvfp4_scale_byte(m1, gc.six_g, gc.y6, gc.fast_b);
-          const float r0 = nvfp4_recip(s0, gc.g), r1 = nvfp4_recip(s1, gc.g);
+          const float r0 = gc.r_tab[s0 & 127u], r1 = gc.r_tab[s1 & 127u];
           if (r0 != 0.0f) c0 = make_uint2(quant8(w[0], w[1], w[2], w[3], r0), quant8(w[4], w[5], w[6], w[7], r0));
           if (r1 != 0.0f) c1 = make_uint2(quant8(w[8], w[9], w[10], w[11], r1), quant8(w[12], w[13], w[14], w[15], r1));
         } else {
@@ -110,7 +127,7 @@ __device__ __forceinline__ void quant_out_row(const QuantOut& q, const QuantOutG
         if (FMT == 0) {
           s0 = nvfp4_scale_byte_f32(m0, gc.six_g, gc.y6, gc.fast_b);
           s1 = nvfp4_scale_byte_f32(m1, gc.six_g, gc.y6, gc.fast_b);
-          const float r0 = nvfp4_recip(s0, gc.g), r1 = nvfp4_recip(s1, gc.g);
+          const float r0 = gc.r_tab[s0 & 127u], r1 = gc.r_tab[s1 & 127u];
           if (r0 != 0.0f) c0 = make_uint2(quant8_f32(lo, r0), quant8_f32(lo + 8, r0));
           if (r1 != 0.0f) c1 = make_uint2(quant8_f32(hi, r1), quant8_f32(hi + 8, r1));
         } else {

@@ -190,6 +190,39 @@ __global__ void __launch_bounds__(kThreads, 4) amax_rot_kernel(const uint4* __re
   }
 }
 
+// The macro-block scaling row pass: one warp per row (grid-stride over the
+// rows), eight 16-byte loads in flight per lane; sigma of the row's largest
+// magnitude.  A non-finite input is reported and clamped as in the DYNAMIC
+// global scale.
+__global__ void __launch_bounds__(kThreads, 4) mbs_rows_kernel(const uint16_t* __restrict__ x,
+                                                               long long rows, int K,
+                                                               float* __restrict__ sigma,
+                                                               unsigned* status) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const long long gwarp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const int n_vec = K / 8;
+  for (long long r = gwarp; r < rows; r += nwarps) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + r * K);
+    unsigned m = 0;
+    for (int v = lane; v < n_vec; v += 256) {
+      uint4 t[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) t[j] = (v + 32 * j < n_vec) ? ld_stream(xr + v + 32 * j) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = max_u16x2(m, mag_max8(t[j]));
+    }
+    m = fold_u16x2(m);
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) {
+      if (m > kBf16MaxFinite) m = amax_checked(m, status);
+      sigma[r] = mbs_sigma(__uint_as_float(m << 16));
+    }
+  }
+}
+
 // -------------------------------------------------------- quantize pass
 
 // n / d for 32-bit n by multiply-high (Granlund & Montgomery, "Division by
@@ -239,7 +272,23 @@ __device__ __forceinline__ void quantize_units(const QuantArgs& a, long long u_b
       unsigned sbyte;
       uint2 packed;
       float r;
-      if (ROT == 0) {
+      if (ROT == 1) {
+        // macro-block scaling (MXFP4): x' = RN(x * RN(1 / sigma_row)), then
+        // the block exponent from the largest |x'| of the lane pair
+        const long long urow = (u < u_end) ? u : u_begin;
+        const long long row =
+            big ? urow / upr : static_cast<long long>(fast_div(static_cast<unsigned>(urow), upr_div));
+        const float rho = __frcp_rn(a.mbs_sigma[row]);
+        float f[16];
+        unpack16(p, q, f);
+        const unsigned long long R = f2(rho, rho);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) f2_split(mul_f2(f2(f[2 * k], f[2 * k + 1]), R), f[2 * k], f[2 * k + 1]);
+        unsigned m = mag_max16(f);
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        sbyte = mxfp4_scale_f32(m, a.rule, &r);
+        packed = make_uint2(quant8_f32(f, r), quant8_f32(f + 8, r));
+      } else if (ROT == 0) {
         unsigned m = fold_u16x2(max_u16x2(mag_max8(p), mag_max8(q)));
         if (FMT == 0) {
           sbyte = nvfp4_scale_byte(m, six_g, y6, fast_b);
@@ -251,7 +300,7 @@ __device__ __forceinline__ void quantize_units(const QuantArgs& a, long long u_b
           sbyte = mxfp4_scale_f32(m << 16, a.rule, &r);
           packed = make_uint2(quant8(p.x, p.y, p.z, p.w, r), quant8(q.x, q.y, q.z, q.w, r));
         }
-      } else {
+      } else if (ROT >= 16) {
         // the unit's rotated values (a 32-value rotation pairs lanes 2i, 2i+1:
         // their units are the two halves of one 32-value block)
         float f[16];
@@ -435,6 +484,12 @@ cudaError_t launch_quantize(const QuantArgs& a_in, cudaStream_t s, bool pdl) {
   const int blocks = static_cast<int>(
       std::max<long long>(1, std::min<long long>(want, static_cast<long long>(sm_count()) * 4)));
   using Kern = void (*)(QuantArgs, long long, int, FastDiv, int, int, long long, long long);
+  if (a.mbs_sigma) {   // MXFP4 with macro-block scaling
+    const Kern k = a.layout == 0 ? quantize_kernel<1, 0, 1> : quantize_kernel<1, 1, 1>;
+    const cudaError_t e =
+        launch_k(k, blocks, pdl, s, a, q.units, q.upr, q.fd, q.nsf, q.ncb, q.pad_a, q.pad_b);
+    return e != cudaSuccess ? e : cudaGetLastError();
+  }
   static const Kern table[3][2][2] = {
       {{quantize_kernel<0, 0, 0>, quantize_kernel<0, 1, 0>},
        {quantize_kernel<1, 0, 0>, quantize_kernel<1, 1, 0>}},
@@ -451,6 +506,19 @@ cudaError_t launch_quantize(const QuantArgs& a_in, cudaStream_t s, bool pdl) {
 }
 
 cudaError_t launch_quantize_act(QuantArgs a, unsigned* partial, cudaStream_t s) {
+  if (a.mbs_sigma) {
+    // the row pass, then the quantize pass (each a programmatic dependent)
+    if (!a.status && !(a.status = watchdog_ptr())) return cudaErrorInvalidSymbol;
+    const long long warps_per_block = kThreads / 32;
+    const int blocks = static_cast<int>(std::max<long long>(
+        1, std::min<long long>((a.rows + warps_per_block - 1) / warps_per_block,
+                               static_cast<long long>(sm_count()) * 4)));
+    cudaError_t e = launch_k(mbs_rows_kernel, blocks, true, s, static_cast<const uint16_t*>(a.x),
+                             a.rows, a.K, a.mbs_sigma, a.status);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_quantize(a, s, true);
+  }
   if (a.dynamic && a.rows * a.K * 2 <= kSelfAmaxBytes) {
     a.self_amax = 1;
     return launch_quantize(a, s, true);

@@ -44,15 +44,17 @@ FP4_MX_RULE_OAS = 1
 
 
 class QuantOpts(ctypes.Structure):
-    """fp4_quant_opts_t: online rotation order (0, 16, 32) and MXFP4 rule."""
-    _fields_ = [("hadamard", ctypes.c_int), ("mx_rule", ctypes.c_int)]
+    """fp4_quant_opts_t: online rotation order (0, 16, 32), MXFP4 rule and
+    the device array that receives the macro-block scales (or NULL)."""
+    _fields_ = [("hadamard", ctypes.c_int), ("mx_rule", ctypes.c_int),
+                ("mbs_scale", ctypes.c_void_p)]
 
 
-def opts(hadamard: int = 0, mx_rule: int = 0):
-    """A fp4_quant_opts_t by reference, or None when both are defaults."""
-    if not hadamard and not mx_rule:
+def opts(hadamard: int = 0, mx_rule: int = 0, mbs_scale=None):
+    """A fp4_quant_opts_t by reference, or None when all are defaults."""
+    if not hadamard and not mx_rule and not mbs_scale:
         return None
-    return ctypes.byref(QuantOpts(hadamard, mx_rule))
+    return ctypes.byref(QuantOpts(hadamard, mx_rule, mbs_scale))
 
 
 class Fp4Error(RuntimeError):
@@ -83,6 +85,7 @@ SIGNATURES = {
     "fp4_gemm_fused": (I, [P, U8P, U8P, FP, I, I, I, I, I, FP, P, I, I, P, SZ, I, P]),
     "fp4_gemm_quant": (I, [U8P, U8P, FP, U8P, U8P, FP, I, I, I, I, I, I, P, FP, U8P, U8P, P, I,
                            P, SZ, I, P]),
+    "fp4_gemm_mbs": (I, [U8P, U8P, FP, U8P, U8P, FP, I, I, I, P, I, I, P, SZ, I, P]),
     "fp4_gemm_grouped": (I, [U8P, U8P, FP, U8P, U8P, FP, P, I, I, I, I, I, P, I, I, P, SZ, I,
                              P]),
     "fp4_gemm_plan": (I, [I, I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
@@ -178,6 +181,12 @@ def fp4_gemm_quant(a_codes, a_scales, g_a, w_codes, w_scales, g_w, M, N, K, fmt,
     return _call("fp4_gemm_quant", a_codes, a_scales, g_a, w_codes, w_scales, g_w, M, N, K, fmt,
                  out_fmt, out_layout, out_opts, g_out, out_codes, out_scales, C, ldc, ws,
                  ws_bytes, max_sms, stream)
+
+
+def fp4_gemm_mbs(a_codes, a_scales, sigma_a, w_codes, w_scales, sigma_w, M, N, K, C, ldc, out, ws,
+                 ws_bytes, max_sms, stream):
+    return _call("fp4_gemm_mbs", a_codes, a_scales, sigma_a, w_codes, w_scales, sigma_w, M, N, K,
+                 C, ldc, out, ws, ws_bytes, max_sms, stream)
 
 
 def fp4_gemm_grouped(a_codes, a_scales, g_a, w_codes, w_scales, g_w, offsets, E, M, N, K, fmt,

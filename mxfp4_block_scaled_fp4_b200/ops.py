@@ -58,11 +58,12 @@ class Quantized:
     K: int
     hadamard: int = 0        # online rotation order (0, 16, 32)
     mx_rule: int = 0         # MXFP4 scale rule (0 OCP, 1 overflow-aware)
+    sigma: torch.Tensor | None = None   # MXFP4 macro-block scales [rows] (or None)
 
 
 def quantize(x: torch.Tensor, fmt: int = NVFP4, layout: int = SCALES_MMA,
              g: torch.Tensor | None = None, ws: torch.Tensor | None = None,
-             hadamard: int = 0, mx_rule: int = 0) -> Quantized:
+             hadamard: int = 0, mx_rule: int = 0, mbs: bool = False) -> Quantized:
     """fp4_quantize_act (fp4_quantize_act_ex with a rotation or rule): DYNAMIC
     global scale when g is None, else STATIC g.  ws: scratch of at least
     fp4_workspace_bytes bytes; calls that may run concurrently (other
@@ -80,20 +81,23 @@ def quantize(x: torch.Tensor, fmt: int = NVFP4, layout: int = SCALES_MMA,
         ws = workspace(ws_bytes, dev)
     elif ws.numel() < ws_bytes:
         raise ValueError("workspace too small")
-    if hadamard or mx_rule:
+    sigma = torch.empty(max(rows, 1), dtype=torch.float32, device=dev) if mbs else None
+    if hadamard or mx_rule or mbs:
         _check(L.fp4_quantize_act_ex(x.data_ptr(), rows, K, fmt, layout, gmode,
-                                     L.opts(hadamard, mx_rule), gt.data_ptr(), codes.data_ptr(),
-                                     scales.data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
+                                     L.opts(hadamard, mx_rule,
+                                            sigma.data_ptr() if mbs else None),
+                                     gt.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                                     ws.data_ptr(), ws.numel(), _stream()),
                "fp4_quantize_act_ex")
     else:
         _check(L.fp4_quantize_act(x.data_ptr(), rows, K, fmt, layout, gmode, gt.data_ptr(),
                                   codes.data_ptr(), scales.data_ptr(), ws.data_ptr(), ws.numel(),
                                   _stream()), "fp4_quantize_act")
-    return Quantized(codes, scales, gt, fmt, layout, rows, K, hadamard, mx_rule)
+    return Quantized(codes, scales, gt, fmt, layout, rows, K, hadamard, mx_rule, sigma)
 
 
 def quantize_weights(w: torch.Tensor, fmt: int = NVFP4, hadamard: int = 0,
-                     mx_rule: int = 0) -> Quantized:
+                     mx_rule: int = 0, mbs: bool = False) -> Quantized:
     """fp4_quantize_weights (fp4_quantize_weights_ex with a rotation or
     rule): one-time, MMA scale layout, DYNAMIC g."""
     _cuda_bf16_2d(w, "w")
@@ -104,8 +108,11 @@ def quantize_weights(w: torch.Tensor, fmt: int = NVFP4, hadamard: int = 0,
                          device=dev)
     g = torch.ones(1, dtype=torch.float32, device=dev)
     ws = workspace(L.fp4_workspace_bytes(N, 0, K, fmt), dev)
-    if hadamard or mx_rule:
-        _check(L.fp4_quantize_weights_ex(w.data_ptr(), N, K, fmt, L.opts(hadamard, mx_rule),
+    sigma = torch.empty(max(N, 1), dtype=torch.float32, device=dev) if mbs else None
+    if hadamard or mx_rule or mbs:
+        _check(L.fp4_quantize_weights_ex(w.data_ptr(), N, K, fmt,
+                                         L.opts(hadamard, mx_rule,
+                                                sigma.data_ptr() if mbs else None),
                                          codes.data_ptr(), scales.data_ptr(), g.data_ptr(),
                                          ws.data_ptr(), ws.numel(), _stream()),
                "fp4_quantize_weights_ex")
@@ -113,7 +120,7 @@ def quantize_weights(w: torch.Tensor, fmt: int = NVFP4, hadamard: int = 0,
         _check(L.fp4_quantize_weights(w.data_ptr(), N, K, fmt, codes.data_ptr(),
                                       scales.data_ptr(), g.data_ptr(), ws.data_ptr(), ws.numel(),
                                       _stream()), "fp4_quantize_weights")
-    return Quantized(codes, scales, g, fmt, SCALES_MMA, N, K, hadamard, mx_rule)
+    return Quantized(codes, scales, g, fmt, SCALES_MMA, N, K, hadamard, mx_rule, sigma)
 
 
 def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
@@ -124,11 +131,19 @@ def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
         raise ValueError("operands must share format and K and use the MMA scale layout")
     if a.hadamard != w.hadamard:
         raise ValueError("a rotated activation needs weights rotated with the same order")
+    if (a.sigma is None) != (w.sigma is None):
+        raise ValueError("macro-block scaling needs both operands quantized with it")
     M, N, K = a.rows, w.rows, a.K
     dev = a.codes.device
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=dev)
     o = L.FP4_OUT_F32 if out.dtype == torch.float32 else L.FP4_OUT_BF16
+    if a.sigma is not None:
+        _check(L.fp4_gemm_mbs(a.codes.data_ptr(), a.scales.data_ptr(), a.sigma.data_ptr(),
+                              w.codes.data_ptr(), w.scales.data_ptr(), w.sigma.data_ptr(), M, N, K,
+                              out.data_ptr(), out.stride(0), o, None, 0, max_sms, _stream()),
+               "fp4_gemm_mbs")
+        return out
     _check(L.fp4_gemm(a.codes.data_ptr(), a.scales.data_ptr(), a.g.data_ptr(),
                       w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(), M, N, K, a.fmt,
                       out.data_ptr(), out.stride(0), o, None, 0, max_sms, _stream()), "fp4_gemm")

@@ -1,0 +1,47 @@
+"""The MMA scale order against an independent consumer: the bytes that
+fp4_quantize_weights / fp4_quantize_act write (packed codes and scales in
+the tensor cores' blocked order) are handed unchanged to the vendor's
+block-scaled FP4 GEMM (cuBLASLt through torch's scaled_mm, 32x4x4 scale
+swizzle), whose result must match the oracle within the bf16 tolerance.
+A layout that this library's own kernels read consistently but that
+differs from the documented blocked order would fail here.  The vendor
+library is used only by this test (and as timing context in bench.py)."""
+import numpy as np
+import pytest
+import torch
+
+from mxfp4_block_scaled_fp4_b200 import inputs
+from tests.parity import gemm_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _scaled_mm():
+    import torch.nn.functional as F
+    need = ("scaled_mm", "ScalingType", "SwizzleType")
+    if not all(hasattr(F, n) for n in need) or not hasattr(torch, "float4_e2m1fn_x2"):
+        pytest.skip("this torch has no block-scaled FP4 scaled_mm")
+    return F
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 1024), (1024, 2048, 4096), (384, 640, 3072)])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_vendor_gemm_reads_our_scale_order(orc, M, N, K, fmt):
+    F = _scaled_mm()
+    from mxfp4_block_scaled_fp4_b200 import ops
+    a = inputs.random_bf16(950 + M, (M, K))
+    w = inputs.random_bf16(951 + N, (N, K), 0.02)
+    aq = ops.quantize(a.cuda(), fmt, ops.SCALES_MMA)
+    wq = ops.quantize_weights(w.cuda(), fmt)
+    sdt = torch.float8_e4m3fn if fmt == 0 else torch.float8_e8m0fnu
+    rec = F.ScalingType.BlockWise1x16 if fmt == 0 else F.ScalingType.BlockWise1x32
+    sw = F.SwizzleType.SWIZZLE_32_4_4
+    c = F.scaled_mm(aq.codes.view(torch.float4_e2m1fn_x2), wq.codes.view(torch.float4_e2m1fn_x2).t(),
+                    aq.scales.view(sdt), rec, wq.scales.view(sdt), rec, sw, sw,
+                    output_dtype=torch.float32)
+    if fmt == 0:
+        c = c * (aq.g * wq.g)            # the vendor call takes no global scales
+    torch.cuda.synchronize()
+    c_ref, _ = orc.w4a4_reference(a, w, fmt)
+    ok, worst, where = gemm_close(c.to(torch.bfloat16), c_ref, torch.bfloat16)
+    assert ok, f"worst err/bound {worst:.3g} at {where}"
