@@ -400,6 +400,13 @@ def measure_vendor(torch, ops, a_dev, w_dev, dev, M, N, K):
             calls = {"ours": lambda: ops.gemm(aq, wq, out=c),
                      "vendor": lambda: F.scaled_mm(A, B, sa, rec, sb, rec, sw, sw,
                                                    output_dtype=torch.bfloat16)}
+            # how far the vendor's result is from ours (it takes no global
+            # scales: NVFP4 is rescaled by g_a g_w), relative to ours' rms
+            ref = ops.gemm(aq, wq, out=c).float()
+            vend = calls["vendor"]().float()
+            if fmt == 0:
+                vend = vend * (aq.g * wq.g)
+            rel = float(((vend - ref).abs().max() / ref.pow(2).mean().sqrt()).item())
             ms = {}
             for key, fn in calls.items():
                 for _ in range(3):
@@ -418,7 +425,8 @@ def measure_vendor(torch, ops, a_dev, w_dev, dev, M, N, K):
             fl = 2.0 * M * N * K
             res[name] = {"ours_tflops": round(fl / ms["ours"] / 1e9, 1),
                          "vendor_tflops": round(fl / ms["vendor"] / 1e9, 1),
-                         "ours_over_vendor": round(ms["vendor"] / ms["ours"], 3)}
+                         "ours_over_vendor": round(ms["vendor"] / ms["ours"], 3),
+                         "vendor_max_diff_over_rms": round(rel, 4)}
         res["vendor"] = "cuBLASLt block-scaled FP4 GEMM via torch.nn.functional.scaled_mm"
         return res
     except Exception as e:  # context only: never fails the bench
@@ -564,7 +572,9 @@ def measure_grouped(torch, ops, dev, fp4_peak):
                          "grouped_tflops": round(flop / res["grouped"] / 1e9, 1),
                          "grouped_frac_fp4_peak": round(flop / res["grouped"] / 1e9 / fp4_peak, 4),
                          "separate_calls_ms": round(res["separate_calls"], 4),
-                         "kernel": "fp4 gemm_kernel grouped (128x128 tiles, device-side offsets)"})
+                         "kernel": ("fp4 gemm_kernel grouped (128x256 tiles" if E <= 128 else
+                                    "fp4 gemm_kernel grouped (128x128 tiles") +
+                                   ", device-side offsets)"})
     st, code = ops.device_status()
     if st != 0:
         raise RuntimeError(f"status word set in the grouped GEMM: {code:#x}")
@@ -612,7 +622,49 @@ def measure_gemm_quant(torch, ops, a, w_dev, dev, fp4_peak):
     return rows
 
 
-def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak):
+def measure_mbs(torch, ops, a, w_dev, dev, fp4_peak):
+    """MXFP4 with macro-block scaling on the largest prefill shape: the GEMM
+    alone (fp4_gemm_mbs) against the plain MXFP4 GEMM, and the activation
+    quantizer (row pass + quantize pass) against the plain one; each call
+    after an L2 flush, median of 20."""
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    Mq, Nq = a.shape[0], w_dev.shape[0]
+    flop = 2.0 * Mq * Nq * K
+    aq_m = ops.quantize(a, 1, ops.SCALES_MMA, mbs=True)
+    wq_m = ops.quantize_weights(w_dev, 1, mbs=True)
+    aq_p = ops.quantize(a, 1, ops.SCALES_MMA)
+    wq_p = ops.quantize_weights(w_dev, 1)
+    c = torch.empty((Mq, Nq), dtype=torch.bfloat16, device=dev)
+    res = {}
+    for name, fn in (("gemm_mbs", lambda: ops.gemm(aq_m, wq_m, out=c)),
+                     ("gemm_plain", lambda: ops.gemm(aq_p, wq_p, out=c)),
+                     ("quantize_mbs", lambda: ops.quantize(a, 1, ops.SCALES_MMA, mbs=True)),
+                     ("quantize_plain", lambda: ops.quantize(a, 1, ops.SCALES_MMA))):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(20):
+            flush_l2(torch, flush, flush_r)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        res[name] = float(np.median(ts))
+    return {"M": Mq, "N": Nq, "K": K, "format": "MXFP4 + per-row macro scales",
+            "gemm_mbs_ms": round(res["gemm_mbs"], 4),
+            "gemm_mbs_tflops": round(flop / res["gemm_mbs"] / 1e9, 1),
+            "gemm_mbs_frac_fp4_peak": round(flop / res["gemm_mbs"] / 1e9 / fp4_peak, 4),
+            "gemm_plain_ms": round(res["gemm_plain"], 4),
+            "quantize_mbs_ms": round(res["quantize_mbs"], 4),
+            "quantize_plain_ms": round(res["quantize_plain"], 4),
+            "note": "quantize_mbs reads the activation twice (row pass + quantize pass)"}
+
+
+def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak, shapes=None):
     """fp4_quantize_act_ex on the activation-quantize sweep, L2 flushed
     before every call: NVFP4 DYNAMIC / STATIC, MXFP4, and the options (the
     online Hadamard rotation of order 16 / 32, the overflow-aware MXFP4
@@ -623,8 +675,25 @@ def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak):
     flush_r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     sp = torch.cuda.current_stream(dev).cuda_stream
     res = []
-    for (M, K) in SWEEP_SHAPES:
+    for (M, K) in (shapes or SWEEP_SHAPES):
         x = inputs.act_sweep(M, K).to(dev)
+        # context: a plain device copy of the same tensor (2 B read + 2 B
+        # written per element), timed the same way -- the bandwidth a tensor
+        # of this size reaches at all, fixed costs included
+        y = torch.empty_like(x)
+        cts = []
+        for i in range(8):
+            flush_l2(torch, flush, flush_r)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            y.copy_(x)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if i >= 3:
+                cts.append(e0.elapsed_time(e1) * 1e3)
+        copy_gbs = 4.0 * M * K / (float(np.median(cts)) * 1e-6) / 1e9
+        del y
         for fmt, gmode, name, had, rule in (
                 (0, 0, "nvfp4_dynamic", 0, 0), (0, 1, "nvfp4_static", 0, 0), (1, 0, "mxfp4", 0, 0),
                 (0, 0, "nvfp4_dynamic_hadamard16", 16, 0), (1, 0, "mxfp4_hadamard32", 32, 0),
@@ -658,6 +727,7 @@ def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak):
                 row["gbs_two_reads"] = round(two / (us * 1e-6) / 1e9, 1)
                 row["frac_hbm_two_reads"] = round(two / (us * 1e-6) / 1e9 / hbm_peak, 4)
             row["frac_hbm_single_pass"] = round(single / (us * 1e-6) / 1e9 / hbm_peak, 4)
+            row["same_size_copy_gbs"] = round(copy_gbs, 1)
             res.append(row)
     return res
 
@@ -729,7 +799,11 @@ def run_part(args, rank):
         peaks_fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16
         line["grouped"] = measure_grouped(torch, ops, dev, peaks_fp4)
     else:
-        line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"])
+        shapes = None
+        if args.quant_shape:
+            shapes = [tuple(int(v) for v in args.quant_shape.split(","))]
+        line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"],
+                                                        shapes)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -767,6 +841,7 @@ def main():
                     choices=["all", "prefill", "decode", "quantize", "decoder", "grouped"],
                     help="run one part only (profiling); the JSON line then carries that part")
     ap.add_argument("--decode-shape", default=None, help="M,N,K: restrict the decode part")
+    ap.add_argument("--quant-shape", default=None, help="M,K: restrict the quantize part")
     ap.add_argument("--shape", default=None,
                     help="M,N,K override (profiling of smaller cases); default 8192,28672,8192")
     args = ap.parse_args()
@@ -974,6 +1049,7 @@ def main():
         line["prefill_matrix"] = measure_prefill_matrix(torch, L, ops, a, w_dev, dev, fp4_peak)
         line["gemm_quant"] = measure_gemm_quant(torch, ops, a, w_dev, dev, fp4_peak)
         line["grouped"] = measure_grouped(torch, ops, dev, fp4_peak)
+        line["mbs"] = measure_mbs(torch, ops, a, w_dev, dev, fp4_peak)
     if not args.no_suite:
         line["decode"] = measure_decode(torch, ops, L, inputs, dev, peaks["hbm_gbs"])
         line["quantize_sweep"] = measure_quantize_sweep(torch, L, inputs, dev, peaks["hbm_gbs"])

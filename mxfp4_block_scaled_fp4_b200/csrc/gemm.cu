@@ -60,6 +60,9 @@ constexpr uint32_t SF_COL = 256;        // per stage: 16 columns A scales + 16 o
 constexpr int kGemmThreads = 352;       // 11 warps: TMA, MMA, 4 epilogue, 4 scale staging, scale TMA
 constexpr int GROUP_M = 16;             // tile raster: 16 M-tiles share their W tiles in L2
 constexpr int kMaxGroups = kGroupedMaxGroups;   // experts of a grouped launch
+// groups a grouped launch of BN-wide tiles can hold (the 256-wide ring
+// leaves room for a table of 128)
+__host__ __device__ constexpr int groups_cap(int bn) { return bn == 256 ? 128 : kMaxGroups; }
 
 // Output tiles are 128 x BN.  BN = 256 is the throughput shape; 128 and 64
 // give problems with few 256-wide tiles more CTAs (and smaller split-K
@@ -79,9 +82,11 @@ struct Tile {
   static constexpr int STAGE_BYTES = A_STAGE + B_STAGE + SFA_BYTES + SFB_STAGE;
   static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128) ? (G ? 5 : 6) : 7;
   static constexpr int RING = STAGES * STAGE_BYTES;
-  static constexpr int GTAB = G ? 4 * (2 * kMaxGroups + 2) : 0;   // group table (ints)
-  static constexpr int SMEM = RING + 1024 + 512 + GTAB + 512;   // ring, alignment, barriers,
-                                                                // groups, reciprocals
+  static constexpr int GCAP = groups_cap(BN);
+  static constexpr int GTAB = G ? 4 * (2 * GCAP + 2) : 0;   // group table (ints)
+  static constexpr int RTAB = G ? 0 : 512;                   // reciprocals of the FP4 epilogue
+  static constexpr int SMEM = RING + 1024 + 512 + GTAB + RTAB;   // ring, alignment, barriers,
+                                                                 // groups, reciprocals
   // tensor-memory columns between the B scales of consecutive atoms, and
   // per stage (A scales in the first 16)
   static constexpr int SFB_ATOM_COLS = 4 * SF_BLOCKS;
@@ -143,9 +148,10 @@ struct GTile {
 // n_tiles); within a group the M tiles are the fastest index, so that
 // consecutive CTAs share a W tile in L2.  gtab: tiles_before[0..E] then the
 // group row starts row0[0..E].
+template <int CAP>
 __device__ __forceinline__ GTile gtile(int t, const Params& p, const int* gtab) {
   const int* before = gtab;
-  const int* row0 = gtab + kMaxGroups + 1;
+  const int* row0 = gtab + CAP + 1;
   int lo = 0, hi = p.E;                         // largest e with before[e] * n_tiles <= t
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -300,14 +306,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (e < p.E) {
           gtab[e] = carry + incl - n;
-          gtab[kMaxGroups + 1 + e] = start;
+          gtab[T::GCAP + 1 + e] = start;
         }
         carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
         prev_end = __shfl_sync(0xFFFFFFFFu, end, 31);
       }
       if (lane == 0) {
         gtab[p.E] = carry;
-        gtab[kMaxGroups + 1 + p.E] = prev_end;
+        gtab[T::GCAP + 1 + p.E] = prev_end;
       }
     }
     __syncthreads();
@@ -335,7 +341,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int t = t_first; t < n_tiles_total; t += t_stride) {
       int mt, nt, a_row0, w_row0;
       if (G) {
-        const GTile g = gtile(t, p, gtab);
+        const GTile g = gtile<T::GCAP>(t, p, gtab);
         nt = g.nt;
         a_row0 = g.a_row0;
         w_row0 = g.e * p.N + nt * BN;
@@ -380,7 +386,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int arb, ablocks = 1;             // A scale row block(s) of the tile
       const uint8_t* wsf = p.w_scales;  // this tile's weight scales
       if (G) {
-        const GTile g = gtile(t, p, gtab);
+        const GTile g = gtile<T::GCAP>(t, p, gtab);
         nt = g.nt;
         arb = g.a_row0 / BM;
         // a tile that does not start on a 128-row boundary spans two blocks
@@ -488,7 +494,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // the stage's two A scale blocks (byte offset; -1 past the tensor)
       int a_word[4] = {0, 0, 0, 0};
       if (G) {
-        const GTile g = gtile(t, p, gtab);
+        const GTile g = gtile<T::GCAP>(t, p, gtab);
         nt = g.nt;
         const int arb = g.a_row0 / BM;
 #pragma unroll
@@ -575,7 +581,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = t_first; t < n_tiles_total; t += t_stride, ++it) {
         int mt, nt, row, row_end = p.M;
         if (G) {
-          const GTile g = gtile(t, p, gtab);
+          const GTile g = gtile<T::GCAP>(t, p, gtab);
           nt = g.nt;
           row = g.a_row0 + quarter * 32 + lane;
           row_end = g.a_row_end;
@@ -975,9 +981,9 @@ cudaError_t launch_gemm_grouped(const GroupedArgs& a, cudaStream_t s) {
   p.a_rowblocks = (a.M + BM - 1) / BM;
   p.splits = 1;
   p.k_per = p.k_steps;
-  // 128 x 128 tiles with all of K (no split): the two A scale blocks a
-  // stage may need leave no room for a 256-wide tile's ring
-  const int bn = 128;
+  // tiles of 128 rows x 256 columns with all of K (no split) when the
+  // table of groups fits beside the 256-wide ring, else 128 x 128
+  const int bn = (a.E <= groups_cap(256) && a.N > 128) ? 256 : 128;
   CUtensorMap ma, mw;
   if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, a.w_codes, static_cast<long long>(a.E) * a.N, a.K, bn))
@@ -985,6 +991,11 @@ cudaError_t launch_gemm_grouped(const GroupedArgs& a, cudaStream_t s) {
   p.n_tiles = (a.N + bn - 1) / bn;
   const long long upper = static_cast<long long>(p.m_tiles) * p.n_tiles;
   const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(upper, sms)));
+  if (bn == 256)
+    return a.fmt == 0 ? (a.out_f32 ? launch_typed<0, 1, 256, 1>(ma, mw, p, grid, s)
+                                   : launch_typed<0, 0, 256, 1>(ma, mw, p, grid, s))
+                      : (a.out_f32 ? launch_typed<1, 1, 256, 1>(ma, mw, p, grid, s)
+                                   : launch_typed<1, 0, 256, 1>(ma, mw, p, grid, s));
   return a.fmt == 0 ? (a.out_f32 ? launch_typed<0, 1, 128, 1>(ma, mw, p, grid, s)
                                  : launch_typed<0, 0, 128, 1>(ma, mw, p, grid, s))
                     : (a.out_f32 ? launch_typed<1, 1, 128, 1>(ma, mw, p, grid, s)
