@@ -692,7 +692,8 @@ def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak, shapes=None):
             torch.cuda.synchronize(dev)
             if i >= 3:
                 cts.append(e0.elapsed_time(e1) * 1e3)
-        copy_gbs = 4.0 * M * K / (float(np.median(cts)) * 1e-6) / 1e9
+        copy_us = float(np.median(cts))
+        copy_gbs = 4.0 * M * K / (copy_us * 1e-6) / 1e9
         del y
         for fmt, gmode, name, had, rule in (
                 (0, 0, "nvfp4_dynamic", 0, 0), (0, 1, "nvfp4_static", 0, 0), (1, 0, "mxfp4", 0, 0),
@@ -728,6 +729,10 @@ def measure_quantize_sweep(torch, L, inputs, dev, hbm_peak, shapes=None):
                 row["frac_hbm_two_reads"] = round(two / (us * 1e-6) / 1e9 / hbm_peak, 4)
             row["frac_hbm_single_pass"] = round(single / (us * 1e-6) / 1e9 / hbm_peak, 4)
             row["same_size_copy_gbs"] = round(copy_gbs, 1)
+            # a copy moves 4 B per element, this pass 2.5 - 4.6: at sizes
+            # where fixed costs dominate both take about the same time
+            row["same_size_copy_us"] = round(copy_us, 3)
+            row["copy_us_over_pass_us"] = round(copy_us / us, 3)
             res.append(row)
     return res
 
