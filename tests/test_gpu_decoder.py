@@ -1,7 +1,8 @@
-"""Synthetic decoder forward (24 layers x 12 W4A4 GEMM calls in the full
-workload; fewer layers here): every recorded call is checked against the
-oracle on the GPU's own inputs (teacher forcing), and the CUDA-graph replay
-must reproduce the eager forward bit for bit."""
+"""Synthetic decoder forward (24 layers x 12 W4A4 GEMM calls): every
+recorded call is checked against the oracle on the GPU's own inputs
+(teacher forcing) -- two layers at M = 1 and 16, all 288 calls of the full
+24-layer forward at M = 1, sampled rows at M = 256 -- and the CUDA-graph
+replay must reproduce the eager forward bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -62,3 +63,19 @@ def test_graph_replay_equals_eager(dec):
     torch.cuda.synchronize()
     assert torch.equal(out, eager)
     assert torch.isfinite(out.float()).all()
+
+
+def test_full_depth_every_call_teacher_forced(orc):
+    """The whole workload's depth: 24 layers, all 288 calls of an M=1
+    forward checked against the oracle on their recorded inputs."""
+    from mxfp4_block_scaled_fp4_b200.decoder import SyntheticDecoder
+    dec24 = SyntheticDecoder("cuda")
+    assert dec24.layers == 24
+    x = torch.randn(1, 2880, generator=torch.Generator().manual_seed(11)).to(torch.bfloat16).cuda()
+    dec24.record = []
+    out = dec24.forward_fp4(x)
+    torch.cuda.synchronize()
+    rec, dec24.record = dec24.record, None
+    assert len(rec) == 288
+    assert torch.isfinite(out.float()).all()
+    _check_calls(orc, dec24, rec)
