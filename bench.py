@@ -510,6 +510,17 @@ def measure_prefill_matrix(torch, L, ops, a_big, w_big, dev, fp4_peak):
 MOE_CONFIGS = [(8, 16384, 4096, 4096), (64, 16384, 2048, 4096)]
 
 
+def grouped_kernel_name(M, N, E, sms=148):
+    """The kernel fp4_gemm_grouped launches for M routed rows over E groups
+    (its launch rule: the CTA-pair form when groups average 512 rows or more
+    and its 256 x 256 tiles keep half the SMs busy)."""
+    pair_ctas = 2 * (-(-M // 256)) * (-(-N // 256))
+    if M >= 512 * E and N > 128 and M > 128 and 2 * pair_ctas >= sms:
+        return "fp4 gemm_pair_kernel grouped (256x256 tiles on CTA pairs"
+    return ("fp4 gemm_kernel grouped (128x256 tiles" if E <= 128 and N > 128 else
+            "fp4 gemm_kernel grouped (128x128 tiles")
+
+
 def measure_grouped(torch, ops, dev, fp4_peak):
     """The grouped (mixture-of-experts) GEMM, fp4_gemm_grouped: E experts of
     [N, K], 16384 routed rows (8192 tokens x 2 experts each) spread over the
@@ -572,9 +583,7 @@ def measure_grouped(torch, ops, dev, fp4_peak):
                          "grouped_tflops": round(flop / res["grouped"] / 1e9, 1),
                          "grouped_frac_fp4_peak": round(flop / res["grouped"] / 1e9 / fp4_peak, 4),
                          "separate_calls_ms": round(res["separate_calls"], 4),
-                         "kernel": ("fp4 gemm_kernel grouped (128x256 tiles" if E <= 128 else
-                                    "fp4 gemm_kernel grouped (128x128 tiles") +
-                                   ", device-side offsets)"})
+                         "kernel": grouped_kernel_name(M, N, E) + ", device-side offsets)"})
     st, code = ops.device_status()
     if st != 0:
         raise RuntimeError(f"status word set in the grouped GEMM: {code:#x}")

@@ -303,11 +303,12 @@ fp4_status_t fp4_gemm_mbs(const uint8_t* a_codes, const uint8_t* a_scales, const
  *               synchronization).  Out-of-range or decreasing entries are
  *               clamped into [0, M] and made non-decreasing, so no row
  *               outside A and C is read or written.
- * 1 <= E <= 256, N % 8 == 0, K % 32 == 0.  Empty groups are allowed.  The
- * tiles are 128 x 128 with all of K (no split), so each element's FP32 sum
- * runs in the same order as fp4_gemm's 128-row kernel.  ws unused (may be
- * NULL).  "FP4 n'existe pas : il existe des FP4, et chaque runtime choisit
- * son dialecte", section "Les runtimes et leurs dialectes : qui parle quoi"
+ * 1 <= E <= 256, N % 8 == 0, K % 32 == 0.  Empty groups are allowed.  Every
+ * tile has all of K (no split): 256 x 256 tiles on CTA pairs when the
+ * groups average at least 512 rows (M >= 512 E), else 128 x 256 tiles
+ * (E <= 128, N > 128) or 128 x 128.  ws unused (may be NULL).
+ * "FP4 n'existe pas : il existe des FP4, et chaque runtime choisit son
+ * dialecte", section "Les runtimes et leurs dialectes : qui parle quoi"
  * (fused NVFP4 MoE kernels, W4A4 MegaMoE). */
 fp4_status_t fp4_gemm_grouped(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
                               const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,

@@ -40,6 +40,7 @@
 #include <cstdio>
 #include <cuda_bf16.h>
 
+#include "groups.cuh"
 #include "internal.h"
 #include "launch_shape.h"
 #include "ptx.cuh"
@@ -60,9 +61,6 @@ constexpr uint32_t SF_COL = 256;        // per stage: 16 columns A scales + 16 o
 constexpr int kGemmThreads = 352;       // 11 warps: TMA, MMA, 4 epilogue, 4 scale staging, scale TMA
 constexpr int GROUP_M = 16;             // tile raster: 16 M-tiles share their W tiles in L2
 constexpr int kMaxGroups = kGroupedMaxGroups;   // experts of a grouped launch
-// groups a grouped launch of BN-wide tiles can hold (the 256-wide ring
-// leaves room for a table of 128)
-__host__ __device__ constexpr int groups_cap(int bn) { return bn == 256 ? 128 : kMaxGroups; }
 
 // Output tiles are 128 x BN.  BN = 256 is the throughput shape; 128 and 64
 // give problems with few 256-wide tiles more CTAs (and smaller split-K
@@ -70,19 +68,19 @@ __host__ __device__ constexpr int groups_cap(int bn) { return bn == 256 ? 128 : 
 // block (two for BN = 256); for BN = 64 the tile is one half of it.  The
 // ring is as deep as shared memory allows, so that narrow tiles keep as
 // many bytes in flight as wide ones.
-// G = 1: the grouped (mixture-of-experts) form, whose A tiles start at any
-// row, so a stage holds the A scale atoms of two 128-row blocks, and the
-// group table follows the barriers.
+// G = 1: the grouped (mixture-of-experts) form: the same ring (a group's
+// tiles start on a 128-row scale block, so a tile's A scales are one
+// block's atoms), and the group table follows the barriers.
 template <int BN, int G = 0>
 struct Tile {
   static constexpr int B_STAGE = BN * BK_BYTES;
   static constexpr int SF_BLOCKS = (BN == 256) ? 2 : 1;
   static constexpr int SFB_STAGE = SF_BLOCKS * 4 * 512;
-  static constexpr int SFA_BYTES = (G ? 2 : 1) * SFA_STAGE;
+  static constexpr int SFA_BYTES = SFA_STAGE;
   static constexpr int STAGE_BYTES = A_STAGE + B_STAGE + SFA_BYTES + SFB_STAGE;
-  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128) ? (G ? 5 : 6) : 7;
+  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128) ? 6 : 7;
   static constexpr int RING = STAGES * STAGE_BYTES;
-  static constexpr int GCAP = groups_cap(BN);
+  static constexpr int GCAP = kMaxGroups;
   static constexpr int GTAB = G ? 4 * (2 * GCAP + 2) : 0;   // group table (ints)
   static constexpr int RTAB = G ? 0 : 512;                   // reciprocals of the FP4 epilogue
   static constexpr int SMEM = RING + 1024 + 512 + GTAB + RTAB;   // ring, alignment, barriers,
@@ -137,34 +135,6 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int
   const int within = t - group * per_group;
   mt = first_m + within % gsize;
   nt = within / gsize;
-}
-
-// A tile of the grouped form: rows [a_row0, a_row_end) of A / C, weight rows
-// from w_row0 of the stacked W, group e.
-struct GTile {
-  int e, a_row0, a_row_end, nt;
-};
-// Tiles of group e occupy [tiles_before[e] * n_tiles, tiles_before[e+1] *
-// n_tiles); within a group the M tiles are the fastest index, so that
-// consecutive CTAs share a W tile in L2.  gtab: tiles_before[0..E] then the
-// group row starts row0[0..E].
-template <int CAP>
-__device__ __forceinline__ GTile gtile(int t, const Params& p, const int* gtab) {
-  const int* before = gtab;
-  const int* row0 = gtab + CAP + 1;
-  int lo = 0, hi = p.E;                         // largest e with before[e] * n_tiles <= t
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (before[mid] * p.n_tiles <= t) lo = mid; else hi = mid;
-  }
-  GTile g;
-  g.e = lo;
-  const int mt_e = before[lo + 1] - before[lo];
-  const int local = t - before[lo] * p.n_tiles;
-  g.nt = local / mt_e;
-  g.a_row0 = row0[lo] + (local - g.nt * mt_e) * BM;
-  g.a_row_end = row0[lo + 1];
-  return g;
 }
 
 // alpha * 8 accumulator values -> 8 bf16 (one 16-byte store) / 2 float4.
@@ -278,44 +248,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (G) {
-    // the group table from the device-side offsets (clamped to [0, M] and
-    // made non-decreasing, so that malformed offsets cannot address rows
-    // outside A and C): warp 0 scans the groups' M-tile counts 32 at a time
-    if (warp == 0) {
-      int carry = 0, prev_end = 0;
-      for (int base = 0; base < p.E; base += 32) {
-        const int e = base + lane;
-        // lanes past the last group repeat its end, so that lane 31 carries
-        // the true end of the groups into the next chunk and the table
-        const int e0 = min(e, p.E);
-        const int r0 = min(max(p.offsets[e0], 0), p.M);
-        const int r1 = (e < p.E) ? min(max(p.offsets[e + 1], 0), p.M) : r0;
-        // non-decreasing starts: a group starts no earlier than the previous end
-        int start = r0;
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xFFFFFFFFu, start, o);
-          if (lane >= o) start = max(start, v);
-        }
-        start = max(start, prev_end);
-        const int end = (e < p.E) ? max(r1, start) : start;
-        int n = (e < p.E) ? (end - start + BM - 1) / BM : 0;
-        int incl = n;
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        if (e < p.E) {
-          gtab[e] = carry + incl - n;
-          gtab[T::GCAP + 1 + e] = start;
-        }
-        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
-        prev_end = __shfl_sync(0xFFFFFFFFu, end, 31);
-      }
-      if (lane == 0) {
-        gtab[p.E] = carry;
-        gtab[T::GCAP + 1 + p.E] = prev_end;
-      }
-    }
+    // the group table from the device-side offsets (groups.cuh)
+    if (warp == 0) build_group_table<T::GCAP>(p.offsets, p.E, p.M, BM, gtab, lane);
     __syncthreads();
     n_tiles_total = gtab[p.E] * p.n_tiles;
   }
@@ -341,7 +275,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int t = t_first; t < n_tiles_total; t += t_stride) {
       int mt, nt, a_row0, w_row0;
       if (G) {
-        const GTile g = gtile<T::GCAP>(t, p, gtab);
+        const GTile g = gtile<T::GCAP>(t, p.E, p.n_tiles, BM, gtab, GROUP_M);
         nt = g.nt;
         a_row0 = g.a_row0;
         w_row0 = g.e * p.N + nt * BN;
@@ -383,14 +317,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t armed = 0, armed_parity = 0;
     for (int t = t_first; t < n_tiles_total; t += t_stride) {
       int mt, nt;
-      int arb, ablocks = 1;             // A scale row block(s) of the tile
+      int arb;                          // A scale row block of the tile
+      const int ablocks = 1;
       const uint8_t* wsf = p.w_scales;  // this tile's weight scales
       if (G) {
-        const GTile g = gtile<T::GCAP>(t, p, gtab);
+        const GTile g = gtile<T::GCAP>(t, p.E, p.n_tiles, BM, gtab, GROUP_M);
         nt = g.nt;
         arb = g.a_row0 / BM;
-        // a tile that does not start on a 128-row boundary spans two blocks
-        ablocks = ((g.a_row0 % BM) != 0 && arb + 1 < p.a_rowblocks) ? 2 : 1;
         wsf += static_cast<long long>(g.e) * p.w_sf_bytes;
       } else {
         tile_coords(t, p, mt, nt);
@@ -490,22 +423,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t phase = 0;
     for (int t = t_first; t < n_tiles_total; t += t_stride) {
       int mt, nt;
-      // G: where tile row i = lane + 32 j of this lane's four words sits in
-      // the stage's two A scale blocks (byte offset; -1 past the tensor)
-      int a_word[4] = {0, 0, 0, 0};
       if (G) {
-        const GTile g = gtile<T::GCAP>(t, p, gtab);
-        nt = g.nt;
-        const int arb = g.a_row0 / BM;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = g.a_row0 + lane + 32 * j;
-          const int blk = r / BM - arb;
-          const int rr = r % BM;
-          a_word[j] = (r / BM < p.a_rowblocks)
-                          ? blk * kAtomsPerStage * 512 + (rr & 31) * 16 + (rr >> 5) * 4
-                          : -1;
-        }
+        nt = gtile<T::GCAP>(t, p.E, p.n_tiles, BM, gtab, GROUP_M).nt;
       } else {
         tile_coords(t, p, mt, nt);
       }
@@ -527,11 +446,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint32_t va[4 * kAtomsPerStage], vb[4 * T::SF_BLOCKS * kAtomsPerStage];
 #pragma unroll
           for (int a = 0; a < kAtomsPerStage; ++a) {
-            if (G) {
-              const uint32_t base = smem_u32(sSFA + stage * SFA_STAGE) + a * 512;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) va[4 * a + j] = a_word[j] >= 0 ? lds32(base + a_word[j]) : 0u;
-            } else {
+            {
               const uint4 x = lds128(sfa_s + a * 512);
               va[4 * a + 0] = x.x; va[4 * a + 1] = x.y; va[4 * a + 2] = x.z; va[4 * a + 3] = x.w;
             }
@@ -579,11 +494,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
       int it = 0;
       for (int t = t_first; t < n_tiles_total; t += t_stride, ++it) {
-        int mt, nt, row, row_end = p.M;
+        int mt, nt, row, row_begin = 0, row_end = p.M;
         if (G) {
-          const GTile g = gtile<T::GCAP>(t, p, gtab);
+          const GTile g = gtile<T::GCAP>(t, p.E, p.n_tiles, BM, gtab, GROUP_M);
           nt = g.nt;
           row = g.a_row0 + quarter * 32 + lane;
+          row_begin = g.a_row_begin;
           row_end = g.a_row_end;
           if (FMT == 0) alpha = __fmul_rn(*p.g_a, p.g_w[g.e]);
         } else {
@@ -595,7 +511,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                p.watchdog, WD_EPILOGUE)))
           break;
         tc_fence_after();
-        const bool row_ok = row < row_end;
+        const bool row_ok = row >= row_begin && row < row_end;
         const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL;
         const float arow = MBS ? __ldg(p.sigma_a + min(row, p.M - 1)) : alpha;
         if (!F32) {
@@ -957,6 +873,10 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
 
 cudaError_t launch_gemm_grouped(const GroupedArgs& a, cudaStream_t s) {
   const int sms = gemm_sms(a.max_sms);
+  // groups of many rows (on average at least two 256-row tiles) take the
+  // CTA-pair form; the offsets stay on the device, so the average decides
+  if (a.M >= 512LL * a.E && a.N > 128 && takes_pair(a.M, a.N, sms))
+    return launch_gemm_pair_grouped(a, s);
   Params p{};
   p.a_scales = a.a_scales;
   p.w_scales = a.w_scales;
@@ -967,9 +887,10 @@ cudaError_t launch_gemm_grouped(const GroupedArgs& a, cudaStream_t s) {
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
-  // M tiles of all groups together: at most one partial tile per group more
-  // than the rows alone need
-  p.m_tiles = (a.M + BM - 1) / BM + a.E;
+  // M tiles of all groups together (a bound for the grid: each group may add
+  // a partial tile at either end, its first one starting on the 128-row
+  // block of its first row)
+  p.m_tiles = (a.M + BM - 1) / BM + 2 * a.E;
   p.k_steps = (a.K + BK - 1) / BK;
   p.ncb = ncb_of(nsf_of(a.K, a.fmt));
   p.w_rowblocks = (a.N + 127) / 128;
@@ -981,9 +902,9 @@ cudaError_t launch_gemm_grouped(const GroupedArgs& a, cudaStream_t s) {
   p.a_rowblocks = (a.M + BM - 1) / BM;
   p.splits = 1;
   p.k_per = p.k_steps;
-  // tiles of 128 rows x 256 columns with all of K (no split) when the
-  // table of groups fits beside the 256-wide ring, else 128 x 128
-  const int bn = (a.E <= groups_cap(256) && a.N > 128) ? 256 : 128;
+  // tiles of 128 rows x 256 columns with all of K (no split); 128 x 128
+  // when N is at most 128
+  const int bn = a.N > 128 ? 256 : 128;
   CUtensorMap ma, mw;
   if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, a.w_codes, static_cast<long long>(a.E) * a.N, a.K, bn))

@@ -47,6 +47,7 @@
 #include <algorithm>
 #include <cuda_bf16.h>
 
+#include "groups.cuh"
 #include "internal.h"
 #include "out_quant.cuh"
 #include "ptx.cuh"
@@ -84,6 +85,18 @@ static_assert(SF_COL + STAGES * SF_STAGE_COLS <= TMEM_COLS, "scale stages exceed
 static_assert(SMEM_BYTES <= 227 * 1024, "ring exceeds shared memory");
 static_assert(RING_BYTES % 1024 == 0, "epilogue buffers must stay 1024-byte aligned");
 
+// The grouped (mixture-of-experts) form, G = 1: the same ring (a group's
+// tiles start on a 128-row scale block, so each CTA half reads one block of
+// A scales, as in the plain form); the group table takes the place of the
+// reciprocals (the grouped form has no FP4 output).
+template <int G>
+struct PairLayout {
+  static constexpr int RTAB = G ? 0 : RTAB_BYTES;
+  static constexpr int GTAB = G ? 4 * (2 * kGroupedMaxGroups + 2) : 0;
+  static constexpr int SMEM = RING_BYTES + OUT_BYTES + RTAB + GTAB + 1024 + 256;
+  static_assert(SMEM <= 227 * 1024, "ring exceeds shared memory");
+};
+
 struct Params {
   const uint8_t* a_scales;
   const uint8_t* w_scales;
@@ -100,6 +113,12 @@ struct Params {
   QuantOut qo;            // OUT 2, 3: the emitted FP4 activation (C optional)
   const float* sigma_a;   // OUT 4, 5: macro-block scales of A rows [M] and W rows [N]
   const float* sigma_w;
+  // grouped form (G = 1): group e is rows [offsets[e], offsets[e+1]) of A
+  // and C and weight rows [e N, e N + N) of the stacked W, whose scales
+  // start at byte e * w_sf_bytes; g_w holds one global scale per group
+  const int* offsets;
+  int E;
+  long long w_sf_bytes;
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int& nt) {
@@ -116,7 +135,7 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int
 // (out_quant.cuh), with the bf16 C stored as well when p.C is not null;
 // 4 / 5 = bf16 / fp32 C scaled by sigma_a[m] sigma_w[n] (MXFP4 macro-block
 // scaling) instead of alpha.
-template <int FMT, int OUT>
+template <int FMT, int OUT, int G = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_w,
@@ -131,8 +150,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sSFA = sB + STAGES * B_STAGE;
   uint8_t* sSFB = sSFA + STAGES * SFA_STAGE;
   uint8_t* sOut = sSFB + STAGES * SFB_STAGE;
-  float* r_tab = reinterpret_cast<float*>(sOut + OUT_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_BYTES + RTAB_BYTES);
+  float* r_tab = reinterpret_cast<float*>(sOut + OUT_BYTES);                          // G = 0
+  int* gtab = reinterpret_cast<int*>(sOut + OUT_BYTES + PairLayout<G>::RTAB);        // G = 1
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_BYTES + PairLayout<G>::RTAB +
+                                               PairLayout<G>::GTAB);
   uint64_t* sf_loaded = full + STAGES;
   uint64_t* empty = sf_loaded + STAGES;
   uint64_t* ready = empty + STAGES;
@@ -175,7 +196,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t peer_abort = map_to_rank(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
 
-  const int n_tiles_total = p.m_tiles * p.n_tiles;
+  int n_tiles_total = p.m_tiles * p.n_tiles;
+  if (G) {
+    // the group table from the device-side offsets (groups.cuh), in both
+    // CTAs of the pair alike
+    if (warp == 0) build_group_table<kGroupedMaxGroups>(p.offsets, p.E, p.M, BM, gtab, lane);
+    __syncthreads();
+    n_tiles_total = gtab[p.E] * p.n_tiles;
+  }
   const int first = static_cast<int>(cluster_id_x());
   const int stride = static_cast<int>(nclusters_x());
   constexpr int kAtomsPerStage = (FMT == 0) ? 4 : 2;
@@ -186,8 +214,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;
     for (int t = first; t < n_tiles_total; t += stride) {
-      int mt, nt;
-      tile_coords(t, p, mt, nt);
+      int a_row, w_row;   // first A row and W row of this CTA's half
+      if (G) {
+        const GTile g = gtile<kGroupedMaxGroups>(t, p.E, p.n_tiles, BM, gtab, GROUP_M);
+        a_row = g.a_row0 + static_cast<int>(rank) * HALF;
+        w_row = g.e * p.N + g.nt * BN + static_cast<int>(rank) * HALF;
+      } else {
+        int mt, nt;
+        tile_coords(t, p, mt, nt);
+        a_row = mt * BM + static_cast<int>(rank) * HALF;
+        w_row = nt * BN + static_cast<int>(rank) * HALF;
+      }
       for (int kb = 0; kb < p.k_steps; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.watchdog, WD_PRODUCER)) {
           st_cluster_u32(peer_abort, 1u);
@@ -195,10 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         {
           mbar_expect_tx(&full[stage], A_STAGE + B_STAGE);
-          tma_load_2d(sA + stage * A_STAGE, &tm_a, kb * BK_BYTES, mt * BM + rank * HALF,
-                      &full[stage]);
-          tma_load_2d(sB + stage * B_STAGE, &tm_w, kb * BK_BYTES, nt * BN + rank * HALF,
-                      &full[stage]);
+          tma_load_2d(sA + stage * A_STAGE, &tm_a, kb * BK_BYTES, a_row, &full[stage]);
+          tma_load_2d(sB + stage * B_STAGE, &tm_w, kb * BK_BYTES, w_row, &full[stage]);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         }
@@ -222,14 +257,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;
     for (int t = first; t < n_tiles_total; t += stride) {
-      int mt, nt;
-      tile_coords(t, p, mt, nt);
-      const int rba = mt * 2 + static_cast<int>(rank);   // A row block of this CTA's half
-      const bool a_rows = rba < p.a_rowblocks;
+      int rba, nt;                     // A scale row block of this CTA's half
+      const uint8_t* wsf = p.w_scales;
+      if (G) {
+        const GTile g = gtile<kGroupedMaxGroups>(t, p.E, p.n_tiles, BM, gtab, GROUP_M);
+        rba = g.a_row0 / HALF + static_cast<int>(rank);
+        nt = g.nt;
+        wsf += static_cast<long long>(g.e) * p.w_sf_bytes;
+      } else {
+        int mt;
+        tile_coords(t, p, mt, nt);
+        rba = mt * 2 + static_cast<int>(rank);
+      }
+      const int ablocks = rba < p.a_rowblocks ? 1 : 0;
       const int rb0 = nt * 2;
       const int wblocks = min(2, p.w_rowblocks - rb0);
       const uint8_t* sfa_g = p.a_scales + static_cast<long long>(rba) * p.ncb * 512;
-      const uint8_t* sfb_g = p.w_scales + static_cast<long long>(rb0) * p.ncb * 512;
+      const uint8_t* sfb_g = wsf + static_cast<long long>(rb0) * p.ncb * 512;
       for (int kb = 0; kb < p.k_steps; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.watchdog, WD_PRODUCER)) {
           st_cluster_u32(peer_abort, 1u);
@@ -241,9 +285,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
           // a half made only of rows past M has no scale atoms; its
           // accumulator rows are never stored
-          mbar_expect_tx(&sf_loaded[stage], sf_bytes * ((a_rows ? 1 : 0) + wblocks));
-          if (a_rows)
-            bulk_load(sSFA + stage * SFA_STAGE, sfa_g + cb0 * 512, sf_bytes, &sf_loaded[stage]);
+          mbar_expect_tx(&sf_loaded[stage], sf_bytes * (ablocks + wblocks));
+          for (int i = 0; i < ablocks; ++i)
+            bulk_load(sSFA + stage * SFA_STAGE + i * kAtomsPerStage * 512,
+                      sfa_g + (static_cast<long long>(i) * p.ncb + cb0) * 512, sf_bytes,
+                      &sf_loaded[stage]);
           for (int i = 0; i < wblocks; ++i)
             bulk_load(sSFB + stage * SFB_STAGE + i * 2048,
                       sfb_g + (static_cast<long long>(i) * p.ncb + cb0) * 512, sf_bytes,
@@ -354,8 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t va[4 * kAtomsPerStage], vb[8 * kAtomsPerStage];
 #pragma unroll
           for (int a = 0; a < kAtomsPerStage; ++a) {
-            const uint4 x = lds128(sfa_s + a * 512);
-            va[4 * a + 0] = x.x; va[4 * a + 1] = x.y; va[4 * a + 2] = x.z; va[4 * a + 3] = x.w;
+            {
+              const uint4 x = lds128(sfa_s + a * 512);
+              va[4 * a + 0] = x.x; va[4 * a + 1] = x.y; va[4 * a + 2] = x.z; va[4 * a + 3] = x.w;
+            }
 #pragma unroll
             for (int rb = 0; rb < 2; ++rb) {
               const uint4 y = lds128(sfb_s + rb * 2048 + a * 512);
@@ -411,17 +459,97 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     int it = 0;
     for (int t = first; t < n_tiles_total; t += stride, ++it) {
-      int mt, nt;
-      tile_coords(t, p, mt, nt);
+      int nt, row0, row_begin = 0, row_end = p.M;   // row0: this warp's first C row
+      if (G) {
+        const GTile g = gtile<kGroupedMaxGroups>(t, p.E, p.n_tiles, BM, gtab, GROUP_M);
+        nt = g.nt;
+        row0 = g.a_row0 + static_cast<int>(rank) * HALF + quarter * 32;
+        row_begin = g.a_row_begin;
+        row_end = g.a_row_end;
+        if (FMT == 0) alpha = __fmul_rn(*p.g_a, p.g_w[g.e]);
+      } else {
+        int mt;
+        tile_coords(t, p, mt, nt);
+        row0 = mt * BM + static_cast<int>(rank) * HALF + quarter * 32;
+      }
+      const int row = row0 + lane;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag,
                                              p.watchdog, WD_EPILOGUE))) {
         if (lane == 0) st_cluster_u32(peer_abort, 1u);
         break;
       }
       tc_fence_after();
-      const int row = mt * BM + static_cast<int>(rank) * HALF + quarter * 32 + lane;
-      const bool row_ok = row < p.M;
+      const bool row_ok = row >= row_begin && row < row_end;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL;
+      if (G && (row0 < row_begin || row0 + 32 > row_end)) {
+        // grouped, a warp whose 32 rows reach outside its group: those rows
+        // belong to the neighbouring groups, so C leaves by per-row stores
+        // of the group's rows only (a TMA store would clip only at 0 and M);
+        // warps inside the group take the TMA-store path below
+        if (!F32) {
+          uint32_t packed[BN / 2];
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r[2 * j])),
+                                                       __fmul_rn(alpha, __uint_as_float(r[2 * j + 1])));
+              packed[16 * c + j] = *reinterpret_cast<uint32_t*>(&h);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader)
+              mbar_arrive(acc_empty);
+            else
+              mbar_arrive_remote(acc_empty_leader);
+          }
+          if (row_ok) {
+            uint16_t* out = static_cast<uint16_t*>(p.C) + static_cast<long long>(row) * p.ldc;
+#pragma unroll
+            for (int v = 0; v < BN / 8; ++v) {
+              const int n = nt * BN + 8 * v;
+              if (n < p.N)
+                *reinterpret_cast<uint4*>(out + n) = make_uint4(packed[4 * v], packed[4 * v + 1],
+                                                                packed[4 * v + 2], packed[4 * v + 3]);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
+            tmem_ld_wait();
+            if (c == BN / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                if (leader)
+                  mbar_arrive(acc_empty);
+                else
+                  mbar_arrive_remote(acc_empty_leader);
+              }
+            }
+            const int n0 = nt * BN + c * 32;
+            if (!row_ok || n0 >= p.N) continue;
+            float* out = static_cast<float*>(p.C) + static_cast<long long>(row) * p.ldc + n0;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              if (n0 + 4 * v < p.N)
+                *reinterpret_cast<float4*>(out + 4 * v) =
+                    make_float4(__fmul_rn(alpha, __uint_as_float(r[4 * v + 0])),
+                                __fmul_rn(alpha, __uint_as_float(r[4 * v + 1])),
+                                __fmul_rn(alpha, __uint_as_float(r[4 * v + 2])),
+                                __fmul_rn(alpha, __uint_as_float(r[4 * v + 3])));
+            }
+          }
+        }
+        continue;
+      }
       // MBS: the row's scale (the column's comes with each value)
       const float arow = MBS ? __ldg(p.sigma_a + min(row, p.M - 1)) : alpha;
       if (!F32) {
@@ -452,7 +580,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // C rows row0 .. row0+31 leave through this warp's two swizzled
         // buffers and 64-column TMA stores (rows past M and columns past N
         // are clipped by the store)
-        const int row0 = mt * BM + static_cast<int>(rank) * HALF + quarter * 32;
         if (row0 < p.M && (!QOUT || p.C != nullptr)) {
 #pragma unroll
           for (int c = 0; c < BN / 64; ++c) {
@@ -488,7 +615,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // by the copy engine instead of 32 scattered 16-byte stores per
         // instruction; the accumulator is released after its last chunk is
         // read
-        const int row0 = mt * BM + static_cast<int>(rank) * HALF + quarter * 32;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
@@ -547,10 +673,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------ host side
 
-template <int FMT, int OUT>
+template <int FMT, int OUT, int G = 0>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc,
                          const Params& p, int tiles, int max_sms, cudaStream_t s) {
-  auto kern = gemm_pair_kernel<FMT, OUT>;
+  auto kern = gemm_pair_kernel<FMT, OUT, G>;
+  constexpr int SMEM_BYTES = PairLayout<G>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -564,7 +691,7 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUt
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // pairs that fit on the device at once (cached per device)
+  // pairs that fit on the device at once (cached per device and form)
   static int max_pairs[64] = {0};
   int dev = 0;
   e = cudaGetDevice(&dev);
@@ -586,6 +713,48 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUt
 }
 
 }  // namespace
+
+cudaError_t launch_gemm_pair_grouped(const GroupedArgs& a, cudaStream_t s) {
+  CUtensorMap ma, mw;
+  if (!make_code_map(&ma, a.a_codes, a.M, a.K, HALF)) return cudaErrorInvalidValue;
+  if (!make_code_map(&mw, a.w_codes, static_cast<long long>(a.E) * a.N, a.K, HALF))
+    return cudaErrorInvalidValue;
+  Params p{};
+  p.a_scales = a.a_scales;
+  p.w_scales = a.w_scales;
+  p.g_a = a.g_a;
+  p.g_w = a.g_w;
+  p.C = a.C;
+  p.ldc = a.ldc;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  // 256-row tiles of all groups together (a bound for the grid: each group
+  // may add a partial tile at either end, its first one starting on the
+  // 128-row block of its first row)
+  p.m_tiles = (a.M + BM - 1) / BM + 2 * a.E;
+  p.n_tiles = (a.N + BN - 1) / BN;
+  p.k_steps = (a.K + BK - 1) / BK;
+  p.ncb = ncb_of(nsf_of(a.K, a.fmt));
+  p.a_rowblocks = (a.M + HALF - 1) / HALF;
+  p.w_rowblocks = (a.N + HALF - 1) / HALF;
+  p.watchdog = watchdog_ptr();
+  if (!p.watchdog) return cudaErrorInvalidSymbol;
+  p.offsets = a.offsets;
+  p.E = a.E;
+  p.w_sf_bytes = static_cast<long long>(p.w_rowblocks) * p.ncb * 512;
+  // C of all groups: warps whose rows lie inside their group store by TMA
+  CUtensorMap mc;
+  if (a.out_f32 ? !make_f32_out_map(&mc, a.C, a.M, a.N, a.ldc, 32)
+                : !make_bf16_out_map(&mc, a.C, a.M, a.N, a.ldc, 32))
+    return cudaErrorInvalidValue;
+  const int tiles = p.m_tiles * p.n_tiles;
+  if (a.fmt == 0)
+    return a.out_f32 ? launch_typed<0, 1, 1>(ma, mw, mc, p, tiles, a.max_sms, s)
+                     : launch_typed<0, 0, 1>(ma, mw, mc, p, tiles, a.max_sms, s);
+  return a.out_f32 ? launch_typed<1, 1, 1>(ma, mw, mc, p, tiles, a.max_sms, s)
+                   : launch_typed<1, 0, 1>(ma, mw, mc, p, tiles, a.max_sms, s);
+}
 
 cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
   CUtensorMap ma, mw, mc;

@@ -134,6 +134,8 @@ struct GroupedArgs {
   int max_sms;
 };
 cudaError_t launch_gemm_grouped(const GroupedArgs& a, cudaStream_t s);
+// Its CTA-pair form (256 x 256 tiles), for groups of many rows.
+cudaError_t launch_gemm_pair_grouped(const GroupedArgs& a, cudaStream_t s);
 
 // Tensor map of packed FP4 codes [rows, K/2] bytes as a 2-D uint8 tensor:
 // box of 128 bytes of K by box_rows rows, 128-byte swizzle, out-of-range

@@ -11,10 +11,14 @@ the shapes of a 2880-hidden / 7680-FFN model:
   => 12 GEMMs per layer, 288 per forward.
 
 Glue between the GEMMs is kept minimal and runs in torch bf16 (it is not
-part of the FP4 path): attention is replaced by passing v through (a
-synthetic stand-in, there is no attention kernel here), the FFN is
-silu(gate) * up, and both sub-blocks are residual with a 1/sqrt(2) scale so
-the activations keep their magnitude over 24 layers without norms.  The
+part of the FP4 path): each sub-block reads an RMS-normalized copy of the
+residual stream (pre-norm, no learned gain), attention is replaced by
+passing v through (a synthetic stand-in, there is no attention kernel here),
+the FFN is silu(gate) * up, and both sub-blocks add back into the residual
+with a 1/sqrt(2) scale.  Without the norms the FFN's product of two
+projections squares the magnitude layer after layer: from the seeded
+weights the bf16 forward overflows to Inf by layer 8 and then turns to NaN;
+with them the residual stream stays near unit RMS over all 24 layers.  The
 split GEMMs write straight into column slices of one output buffer (ldc =
 the full width), so no concatenation runs.  Every GEMM call goes through
 the library: fp4_gemm_fused for M <= 32 (activation quantized inside the
@@ -52,6 +56,12 @@ LAYER_GEMMS = ([("q", HIDDEN, HIDDEN), ("k", HIDDEN, HIDDEN), ("v", HIDDEN, HIDD
                [(f"up{i}", FFN // 2, HIDDEN) for i in range(2)] +
                [(f"down{i}", HIDDEN // 4, FFN) for i in range(4)])
 RES = 1.0 / math.sqrt(2.0)
+
+
+def _norm(x: torch.Tensor) -> torch.Tensor:
+    """Pre-norm of a sub-block's input: RMS normalization over the hidden
+    dimension, no learned gain (torch glue, bf16)."""
+    return torch.nn.functional.rms_norm(x, (x.shape[-1],))
 
 
 class SyntheticDecoder:
@@ -139,15 +149,17 @@ class SyntheticDecoder:
             tq = torch.empty((M, HIDDEN), dtype=bf, device=dev)
             tk = torch.empty((M, HIDDEN), dtype=bf, device=dev)
             v = torch.empty((M, HIDDEN), dtype=bf, device=dev)
-            self._branches([lambda: self._gemm(li, "v", x, v),
-                            lambda: self._gemm(li, "q", x, tq),
-                            lambda: self._gemm(li, "k", x, tk)])
+            xn = _norm(x)
+            self._branches([lambda: self._gemm(li, "v", xn, v),
+                            lambda: self._gemm(li, "q", xn, tq),
+                            lambda: self._gemm(li, "k", xn, tk)])
             o = self._gemm(li, "o", v, torch.empty((M, HIDDEN), dtype=bf, device=dev))
             x = (x + o) * RES
             gate = torch.empty((M, FFN), dtype=bf, device=dev)
             up = torch.empty((M, FFN), dtype=bf, device=dev)
             half = FFN // 2
-            self._branches([lambda i=i, t=t, name=name: self._gemm(li, f"{name}{i}", x,
+            xn = _norm(x)
+            self._branches([lambda i=i, t=t, name=name: self._gemm(li, f"{name}{i}", xn,
                                                                    t[:, i * half:(i + 1) * half])
                             for name, t in (("gate", gate), ("up", up)) for i in range(2)])
             h = torch.nn.functional.silu(gate) * up
@@ -162,10 +174,12 @@ class SyntheticDecoder:
     def forward_bf16(self, x: torch.Tensor) -> torch.Tensor:
         for li in range(self.layers):
             W = self.wb[li]
-            v, _, _ = self._branches([lambda: x @ W["v"].T, lambda: x @ W["q"].T,
-                                      lambda: x @ W["k"].T])
+            xn = _norm(x)
+            v, _, _ = self._branches([lambda: xn @ W["v"].T, lambda: xn @ W["q"].T,
+                                      lambda: xn @ W["k"].T])
             x = (x + v @ W["o"].T) * RES
-            g, u = self._branches([lambda: x @ W["gate"].T, lambda: x @ W["up"].T])
+            xn = _norm(x)
+            g, u = self._branches([lambda: xn @ W["gate"].T, lambda: xn @ W["up"].T])
             h = torch.nn.functional.silu(g) * u
             x = (x + h @ W["down"].T) * RES
         return x

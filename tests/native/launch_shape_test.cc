@@ -22,6 +22,16 @@ void expect(int m_tiles, int N, int k_steps, int sms, int bn, int splits) {
   }
 }
 
+// the FP4-emitting and macro-block-scaled epilogues take no K split
+void expect_nosplit(int m_tiles, int N, int k_steps, int sms, int bn) {
+  const fp4::Shape s = fp4::choose_shape(m_tiles, N, k_steps, sms, clusters_148, false);
+  if (s.bn != bn || s.splits != 1) {
+    std::printf("no split: m_tiles=%d N=%d k_steps=%d sms=%d: got %dx%d, expected %dx1\n",
+                m_tiles, N, k_steps, sms, s.bn, s.splits, bn);
+    ++failures;
+  }
+}
+
 void expect_pair(int M, int N, int sms, bool pair) {
   if (fp4::takes_pair(M, N, sms) != pair) {
     std::printf("M=%d N=%d sms=%d: pair %d, expected %d\n", M, N, sms, !pair, pair);
@@ -52,6 +62,11 @@ int main() {
   expect(2, 2880, 12, 49, 128, 1);
   expect(2, 3840, 12, 37, 256, 1);
   expect(2, 720, 30, 37, 128, 2);
+  // without a K split the few-tile shapes keep their narrowest one-wave tile
+  expect_nosplit(2, 720, 30, 148, 64);     // split 5 above
+  expect_nosplit(2, 2880, 30, 148, 64);    // split 2 above
+  expect_nosplit(1, 720, 30, 148, 64);
+  expect_nosplit(2, 2880, 12, 148, 64);    // unchanged (no split above either)
   // the CTA-pair kernel
   expect_pair(8192, 28672, 148, true);
   expect_pair(600, 4104, 148, true);

@@ -76,6 +76,14 @@ def test_grouped_matches_oracle(ops, orc, E, M, N, K, fmt, dt):
     _run(ops, orc, E, M, N, K, fmt, dt, seed=E + M)
 
 
+# groups of many rows on average take the CTA-pair form (256 x 256 tiles)
+@pytest.mark.parametrize("E,M,N,K", [(4, 4096, 2048, 1024), (8, 8192, 1536, 768)])
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_grouped_pair_form_matches_oracle(ops, orc, E, M, N, K, fmt, dt):
+    _run(ops, orc, E, M, N, K, fmt, dt, seed=E + M + 1)
+
+
 def test_groups_of_one_row_and_empty_tail(ops, orc):
     sizes = np.array([1, 0, 1, 129, 0, 127, 1, 0], np.int64)
     _run(ops, orc, 8, int(sizes.sum()), 384, 512, 0, "bf16", seed=5, sizes=sizes)
@@ -109,6 +117,29 @@ def test_malformed_offsets_are_clamped(ops, orc):
             one = ops.Quantized(wq.codes[e], wq.scales[e], wq.g[e:e + 1], 0, ops.SCALES_MMA, N, K)
             ref[lo:hi] = ops.gemm(sub, one, torch.float32).cpu()
     torch.cuda.synchronize()
+    got = c.cpu()
+    assert torch.allclose(got, ref, rtol=1e-4, atol=1e-4 * float(ref.abs().max()))
+
+
+def test_malformed_offsets_pair_form(ops, orc):
+    """The same clamping on the CTA-pair form."""
+    M, N, K, E = 4096, 1024, 512, 4
+    a = inputs.random_bf16(720, (M, K)).cuda()
+    w = inputs.random_bf16(721, (E * N, K), 0.02).view(E, N, K).cuda().contiguous()
+    aq = ops.quantize(a, 0, ops.SCALES_MMA)
+    wq = ops.quantize_experts(w, 0)
+    offs = torch.tensor([-50, 1000, 900, 3000, 99_999], dtype=torch.int32, device="cuda")
+    c = torch.full((M, N), 7.0, dtype=torch.float32, device="cuda")
+    ops.gemm_grouped(aq, wq, offs, out=c)
+    torch.cuda.synchronize()
+    st, code = ops.device_status()
+    assert st == 0 and code == 0
+    ref = torch.full((M, N), 7.0, dtype=torch.float32)
+    for e, (lo, hi) in enumerate([(0, 1000), (1000, 1000), (1000, 3000), (3000, 4096)]):
+        if hi > lo:
+            sub = ops.quantize(a[lo:hi].contiguous(), 0, ops.SCALES_MMA, g=aq.g)
+            one = ops.Quantized(wq.codes[e], wq.scales[e], wq.g[e:e + 1], 0, ops.SCALES_MMA, N, K)
+            ref[lo:hi] = ops.gemm(sub, one, torch.float32).cpu()
     got = c.cpu()
     assert torch.allclose(got, ref, rtol=1e-4, atol=1e-4 * float(ref.abs().max()))
 
