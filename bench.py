@@ -117,18 +117,23 @@ class Clocks:
             try:
                 sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
                 rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.samples.append((sm, smax, rs))
+                self.samples.append((time.perf_counter(), sm, smax, rs))
             except Exception as e:  # keep the region's timing intact
                 self.nvml_err = str(e)[:80]
                 return
             time.sleep(0.001)
 
     def start(self):
+        """Starts the samplers and returns once the NVML thread is taking
+        samples (its first calls can take longer than a short region)."""
         import threading
         try:
             h = self._handle()
             self.thread = threading.Thread(target=self._loop, args=(h,), daemon=True)
             self.thread.start()
+            t_end = time.perf_counter() + 2.0
+            while not self.samples and self.nvml_err is None and time.perf_counter() < t_end:
+                time.sleep(0.001)
         except Exception as e:
             self.nvml_err = f"{type(e).__name__}: {str(e)[:80]}"
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -140,6 +145,7 @@ class Clocks:
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        self.t0 = time.perf_counter()
 
     def _smi(self):
         if self.proc is None:
@@ -165,16 +171,27 @@ class Clocks:
         return rows
 
     def stop(self):
+        """Summary of the samples taken between start() and stop(); a region
+        shorter than one NVML round trip gets the first sample after it."""
+        t1 = time.perf_counter()
+        if self.thread is not None:
+            t_end = t1 + 0.1
+            while (not any(t > t1 for t, *_ in self.samples) and self.nvml_err is None
+                   and time.perf_counter() < t_end):
+                time.sleep(0.001)
         self.stop_flag = True
         if self.thread is not None:
             self.thread.join(timeout=5)
         smi = self._smi()
+        inside = [x for x in self.samples if self.t0 <= x[0] <= t1]
+        after = [x for x in self.samples if x[0] > t1][:1]
+        picked = inside or after
         reasons, sm, smax = set(), [], None
-        for mhz, mx, rs in self.samples:
+        for _, mhz, mx, rs in picked:
             sm.append(float(mhz))
             smax = float(mx)
             reasons |= {nm for nm, bit in self.REASONS if rs & bit}
-        source = "nvml 1 ms"
+        source = "nvml 1 ms" if inside else "nvml, first sample after the region"
         if not sm:
             source = "nvidia-smi 200 ms"
             for mhz, mx, rs in smi:

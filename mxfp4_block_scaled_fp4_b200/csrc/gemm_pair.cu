@@ -92,8 +92,11 @@ static_assert(RING_BYTES % 1024 == 0, "epilogue buffers must stay 1024-byte alig
 template <int G>
 struct PairLayout {
   static constexpr int RTAB = G ? 0 : RTAB_BYTES;
+  // macro-block scaling (OUT 4, 5): the tile's 256 column scales, double
+  // buffered across tiles
+  static constexpr int SIGW = G ? 0 : 2 * BN * 4;
   static constexpr int GTAB = G ? 4 * (2 * kGroupedMaxGroups + 2) : 0;
-  static constexpr int SMEM = RING_BYTES + OUT_BYTES + RTAB + GTAB + 1024 + 256;
+  static constexpr int SMEM = RING_BYTES + OUT_BYTES + RTAB + SIGW + GTAB + 1024 + 256;
   static_assert(SMEM <= 227 * 1024, "ring exceeds shared memory");
 };
 
@@ -151,16 +154,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sSFB = sSFA + STAGES * SFA_STAGE;
   uint8_t* sOut = sSFB + STAGES * SFB_STAGE;
   float* r_tab = reinterpret_cast<float*>(sOut + OUT_BYTES);                          // G = 0
-  int* gtab = reinterpret_cast<int*>(sOut + OUT_BYTES + PairLayout<G>::RTAB);        // G = 1
+  float* sigw = reinterpret_cast<float*>(sOut + OUT_BYTES + PairLayout<G>::RTAB);     // G = 0
+  int* gtab = reinterpret_cast<int*>(sOut + OUT_BYTES + PairLayout<G>::RTAB +
+                                     PairLayout<G>::SIGW);                           // G = 1
   uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_BYTES + PairLayout<G>::RTAB +
-                                               PairLayout<G>::GTAB);
+                                               PairLayout<G>::SIGW + PairLayout<G>::GTAB);
   uint64_t* sf_loaded = full + STAGES;
   uint64_t* empty = sf_loaded + STAGES;
   uint64_t* ready = empty + STAGES;
   uint64_t* acc_full = ready + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sw_ready = drain + 1;   // MBS: the two column-scale buffers (4 epilogue warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sw_ready + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -178,6 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);       // 4 epilogue warps in each CTA of the pair
     mbar_init(drain, 1);
+    mbar_init(&sw_ready[0], 4);
+    mbar_init(&sw_ready[1], 4);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm_a);
@@ -473,6 +481,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         row0 = mt * BM + static_cast<int>(rank) * HALF + quarter * 32;
       }
       const int row = row0 + lane;
+      // MBS: the tile's column scales into shared memory while the MMAs run
+      // (a tile's epilogue reads each of them 128 times per CTA), each warp a
+      // quarter of them; the buffer alternates between tiles, and a warp
+      // passes the (bounded) wait of tile t + 1 only after every epilogue
+      // warp has arrived for it, i.e. has finished tile t - 1
+      float* sw = sigw + (it & 1) * BN;
+      if (MBS) {
+        for (int j = threadIdx.x - 64; j < BN; j += 128) {
+          const int n = nt * BN + j;
+          sw[j] = n < p.N ? __ldg(p.sigma_w + n) : 0.0f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sw_ready[it & 1]);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sw_ready[it & 1], static_cast<uint32_t>(it >> 1) & 1u,
+                                               abort_flag, p.watchdog, WD_EPILOGUE))) {
+          if (lane == 0) st_cluster_u32(peer_abort, 1u);
+          break;
+        }
+      }
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag,
                                              p.watchdog, WD_EPILOGUE))) {
         if (lane == 0) st_cluster_u32(peer_abort, 1u);
@@ -561,10 +588,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = nt * BN + 32 * c + 2 * j;
-            const float lo = __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n, p.N), __uint_as_float(r[2 * j]));
+            const int jc = 32 * c + 2 * j;   // column within the tile
+            const float lo = __fmul_rn(MBS ? __fmul_rn(arow, sw[jc]) : arow, __uint_as_float(r[2 * j]));
             const float hi =
-                __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 1, p.N), __uint_as_float(r[2 * j + 1]));
+                __fmul_rn(MBS ? __fmul_rn(arow, sw[jc + 1]) : arow, __uint_as_float(r[2 * j + 1]));
             __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
             packed[16 * c + j] = *reinterpret_cast<uint32_t*>(&h);
           }
@@ -639,12 +666,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t rowaddr = smem_u32(buf) + lane * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int n = n0 + 4 * j;
+            const int jc = c * 32 + 4 * j;   // column within the tile
             sts128(rowaddr + ((j ^ (lane & 7)) << 4),
-                   __float_as_uint(__fmul_rn(col_scale<MBS>(arow, p.sigma_w, n, p.N), __uint_as_float(r[4 * j + 0]))),
-                   __float_as_uint(__fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 1, p.N), __uint_as_float(r[4 * j + 1]))),
-                   __float_as_uint(__fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 2, p.N), __uint_as_float(r[4 * j + 2]))),
-                   __float_as_uint(__fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 3, p.N), __uint_as_float(r[4 * j + 3]))));
+                   __float_as_uint(__fmul_rn(MBS ? __fmul_rn(arow, sw[jc]) : arow, __uint_as_float(r[4 * j + 0]))),
+                   __float_as_uint(__fmul_rn(MBS ? __fmul_rn(arow, sw[jc + 1]) : arow, __uint_as_float(r[4 * j + 1]))),
+                   __float_as_uint(__fmul_rn(MBS ? __fmul_rn(arow, sw[jc + 2]) : arow, __uint_as_float(r[4 * j + 2]))),
+                   __float_as_uint(__fmul_rn(MBS ? __fmul_rn(arow, sw[jc + 3]) : arow, __uint_as_float(r[4 * j + 3]))));
           }
           fence_proxy_async_smem();
           __syncwarp();

@@ -94,6 +94,14 @@ def test_max_groups(ops, orc):
     _run(ops, orc, 256, 768, 128, 256, 0, "f32", seed=6, sizes=sizes)
 
 
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_max_groups_wide_tiles(ops, orc, fmt):
+    """256 groups with N > 128: 128 x 256 tiles beside a full group table;
+    groups of 1 to 9 rows, so most start inside a 128-row scale block."""
+    sizes = (np.arange(256, dtype=np.int64) % 9) + 1
+    _run(ops, orc, 256, int(sizes.sum()), 384, 512, fmt, "f32", seed=7, sizes=sizes)
+
+
 def test_malformed_offsets_are_clamped(ops, orc):
     """Decreasing and out-of-range entries: the kernel clamps them into
     [0, M], keeps the groups disjoint and leaves every other row alone."""
