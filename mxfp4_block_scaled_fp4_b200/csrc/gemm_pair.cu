@@ -142,7 +142,8 @@ template <int FMT, int OUT, int G = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_w,
-                     const __grid_constant__ CUtensorMap tm_c, const Params p) {
+                     const __grid_constant__ CUtensorMap tm_c,
+                     const __grid_constant__ CUtensorMap tm_q, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   // the same 1024-aligned offset in both CTAs: the pair MMA addresses the
   // peer's operands with this CTA's descriptors
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_w);
     if (!(OUT == 2 || OUT == 3) || p.C != nullptr) prefetch_tensormap(&tm_c);
+    if (OUT == 2 || OUT == 3) prefetch_tensormap(&tm_q);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -632,8 +634,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (QOUT) {
+          // the codes of rows row0 .. row0+31 (128 bytes each) leave through
+          // this warp's second buffer and one TMA store (rows past M and
+          // bytes past N / 2 are clipped by the store); the scales by word
+          // stores.  (The next tile's first C chunk uses the first buffer,
+          // and its second chunk waits for this store as for any other.)
           const bool pad = p.qo.layout == 0 && !row_ok && row < p.a_rowblocks * HALF;
-          quant_out_row<BN, QOUT ? OUT - 2 : 0>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N);
+          uint8_t* qbuf = sOutW + OUT_BUF;
+          if (lane == 0) bulk_wait_read_0();   // every earlier store has read its buffer
+          __syncwarp();
+          const uint32_t srow = row0 < p.M ? smem_u32(qbuf) + lane * 128 : 0u;
+          quant_out_row<BN, QOUT ? OUT - 2 : 0>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N,
+                                                srow, lane & 7);
+          if (row0 < p.M) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_q, qbuf, nt * (BN / 2), row0);
+              bulk_commit();
+            }
+          }
         }
       } else {
         // fp32: 32-column chunks leave through the warp's two swizzled
@@ -702,6 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int FMT, int OUT, int G = 0>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc,
+                         const CUtensorMap& mq,
                          const Params& p, int tiles, int max_sms, cudaStream_t s) {
   auto kern = gemm_pair_kernel<FMT, OUT, G>;
   constexpr int SMEM_BYTES = PairLayout<G>::SMEM;
@@ -734,7 +755,7 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUt
   }
   const int pairs = std::max(1, std::min({tiles, max_pairs[dev], gemm_sms(max_sms) / 2}));
   cfg.gridDim = dim3(2 * pairs);
-  e = cudaLaunchKernelEx(&cfg, kern, ma, mw, mc, p);
+  e = cudaLaunchKernelEx(&cfg, kern, ma, mw, mc, mq, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -777,21 +798,28 @@ cudaError_t launch_gemm_pair_grouped(const GroupedArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   const int tiles = p.m_tiles * p.n_tiles;
   if (a.fmt == 0)
-    return a.out_f32 ? launch_typed<0, 1, 1>(ma, mw, mc, p, tiles, a.max_sms, s)
-                     : launch_typed<0, 0, 1>(ma, mw, mc, p, tiles, a.max_sms, s);
-  return a.out_f32 ? launch_typed<1, 1, 1>(ma, mw, mc, p, tiles, a.max_sms, s)
-                   : launch_typed<1, 0, 1>(ma, mw, mc, p, tiles, a.max_sms, s);
+    return a.out_f32 ? launch_typed<0, 1, 1>(ma, mw, mc, ma, p, tiles, a.max_sms, s)
+                     : launch_typed<0, 0, 1>(ma, mw, mc, ma, p, tiles, a.max_sms, s);
+  return a.out_f32 ? launch_typed<1, 1, 1>(ma, mw, mc, ma, p, tiles, a.max_sms, s)
+                   : launch_typed<1, 0, 1>(ma, mw, mc, ma, p, tiles, a.max_sms, s);
 }
 
 cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
-  CUtensorMap ma, mw, mc;
+  CUtensorMap ma, mw, mc, mq;
   if (!make_code_map(&ma, a.a_codes, a.M, a.K, HALF)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, a.w_codes, a.N, a.K, HALF)) return cudaErrorInvalidValue;
   const bool f32 = a.out_mode == 1 || a.out_mode == 5;
-  if ((a.out_mode == 2 || a.out_mode == 3) && !a.C)
+  const bool qout = a.out_mode == 2 || a.out_mode == 3;
+  if (qout && !a.C)
     mc = ma;   // unused: no bf16 C beside the FP4 output
   else if (f32 ? !make_f32_out_map(&mc, a.C, a.M, a.N, a.ldc, 32)
                : !make_bf16_out_map(&mc, a.C, a.M, a.N, a.ldc, 32))
+    return cudaErrorInvalidValue;
+  // the emitted codes [M, N / 2]: 128-byte x 32-row boxes, one per epilogue
+  // warp and tile (unused otherwise)
+  if (!qout)
+    mq = ma;
+  else if (!make_code_map(&mq, a.qo.codes, a.M, a.N, 32))
     return cudaErrorInvalidValue;
   Params p;
   p.a_scales = a.a_scales;
@@ -816,16 +844,16 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
   p.sigma_w = a.sigma_w;
   const int tiles = p.m_tiles * p.n_tiles;
   using L = cudaError_t (*)(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                            const Params&, int, int, cudaStream_t);
+                            const CUtensorMap&, const Params&, int, int, cudaStream_t);
   static const L table[2][4] = {
       {launch_typed<0, 0>, launch_typed<0, 1>, launch_typed<0, 2>, launch_typed<0, 3>},
       {launch_typed<1, 0>, launch_typed<1, 1>, launch_typed<1, 2>, launch_typed<1, 3>}};
   if (a.out_mode >= 4) {   // macro-block scaling: MXFP4 only
     if (a.fmt != 1) return cudaErrorInvalidValue;
-    return a.out_mode == 5 ? launch_typed<1, 5>(ma, mw, mc, p, tiles, a.max_sms, s)
-                           : launch_typed<1, 4>(ma, mw, mc, p, tiles, a.max_sms, s);
+    return a.out_mode == 5 ? launch_typed<1, 5>(ma, mw, mc, ma, p, tiles, a.max_sms, s)
+                           : launch_typed<1, 4>(ma, mw, mc, ma, p, tiles, a.max_sms, s);
   }
-  return table[a.fmt != 0][a.out_mode](ma, mw, mc, p, tiles, a.max_sms, s);
+  return table[a.fmt != 0][a.out_mode](ma, mw, mc, mq, p, tiles, a.max_sms, s);
 }
 
 }  // namespace fp4

@@ -81,10 +81,14 @@ __device__ __forceinline__ void rotate32_in_thread(float lo[16], float hi[16], f
 // a row of the last 128-row block past M (MMA order) gets zero scales.
 // Scale columns past N up to the 4-column group boundary (MMA order) are
 // written as zero by the tile that covers them.  N % 32 == 0.
+// srow != 0: the row's BN / 2 code bytes go to shared memory at srow (16-byte
+// chunk j at srow + ((j ^ swz) << 4), the 128-byte swizzle of a TMA store
+// box) instead of global memory; the caller stores the box.
 template <int BN, int FMT>
 __device__ __forceinline__ void quant_out_row(const QuantOut& q, const QuantOutG& gc,
                                               const uint32_t* packed, long long row, bool row_real,
-                                              bool row_pad, int n0, int N) {
+                                              bool row_pad, int n0, int N, uint32_t srow = 0u,
+                                              int swz = 0) {
   constexpr int B16 = BN / 16;
   if (!row_real && !row_pad) return;
   uint8_t sb[B16];
@@ -137,8 +141,12 @@ __device__ __forceinline__ void quant_out_row(const QuantOut& q, const QuantOutG
           c1 = make_uint2(quant8_f32(hi, r), quant8_f32(hi + 8, r));
         }
       }
-      *reinterpret_cast<uint4*>(q.codes + row * (N / 2) + col / 2) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+      if (srow == 0u)
+        *reinterpret_cast<uint4*>(q.codes + row * (N / 2) + col / 2) = make_uint4(c0.x, c0.y, c1.x, c1.y);
     }
+    if (srow != 0u)
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(srow + (((u >> 1) ^ swz) << 4)),
+                   "r"(c0.x), "r"(c0.y), "r"(c1.x), "r"(c1.y) : "memory");
     sb[u] = static_cast<uint8_t>(s0);
     sb[u + 1] = static_cast<uint8_t>(s1);
   }
@@ -149,6 +157,25 @@ __device__ __forceinline__ void quant_out_row(const QuantOut& q, const QuantOutG
   const int c0 = FMT == 0 ? n0 / 16 : n0 / 32;
   const int c_end = q.layout == 0 ? 4 * q.ncb : q.nsf;   // padding columns up to the group
   if (!row_real && q.layout != 0) return;
+  // four consecutive scale columns from a multiple of 4 are one aligned word
+  // in the MMA order (and in a row-major order whose rows are whole words):
+  // one 4-byte store instead of four byte stores
+  if (per % 4 == 0 && (q.layout == 0 || q.nsf % 4 == 0)) {
+#pragma unroll
+    for (int j = 0; j < per; j += 4) {
+      const int c = c0 + j;
+      if (c >= c_end) break;
+      uint32_t v = 0u;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (row_real && c + k < q.nsf) v |= static_cast<uint32_t>(FMT == 0 ? sb[j + k] : sb[2 * (j + k)]) << (8 * k);
+      *reinterpret_cast<uint32_t*>(q.scales + out_scale_offset(q, row, c)) = v;
+    }
+    if (n0 + BN >= N)
+      for (int c = c0 + per; c < c_end; c += 4)
+        *reinterpret_cast<uint32_t*>(q.scales + out_scale_offset(q, row, c)) = 0u;
+    return;
+  }
 #pragma unroll
   for (int j = 0; j < per; ++j) {
     const int c = c0 + j;
