@@ -168,21 +168,17 @@ __device__ __forceinline__ unsigned long long fma_f2(unsigned long long a, unsig
   return r;
 }
 
-// The in-unit stages h = 1, 2, 4, 8 of the transform, then (n = 16) the
-// scaling; n = 32 adds the cross-lane stage h = 16 (every lane of the warp
-// must take part) before it.  `odd` = this unit is the upper half of its
-// 32-value block.  Stage h = 1 pairs the two lanes of a packed register
-// (scalar adds); from h = 2 on a pair of registers (i, i + h) moves as one
-// packed add and one packed subtract.
-template <int N>
-__device__ __forceinline__ void rotate_unit(float f[16], float scale, bool odd) {
+// The in-unit stages h = 1, 2, 4, 8 of the transform on 16 values, left as
+// 8 packed pairs (P[k] = values 2k, 2k+1).  Stage h = 1 pairs the two lanes
+// of a packed register (scalar adds); from h = 2 on a pair of registers
+// (i, i + h) moves as one packed add and one packed subtract.
+__device__ __forceinline__ void fwht16_packed(float f[16], unsigned long long P[8]) {
 #pragma unroll
   for (int i = 0; i < 16; i += 2) {
     const float a = f[i], b = f[i + 1];
     f[i] = __fadd_rn(a, b);
     f[i + 1] = __fsub_rn(a, b);
   }
-  unsigned long long P[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) P[k] = f2(f[2 * k], f[2 * k + 1]);
 #pragma unroll
@@ -196,6 +192,15 @@ __device__ __forceinline__ void rotate_unit(float f[16], float scale, bool odd) 
       }
     }
   }
+}
+
+// The stages h = 1, 2, 4, 8 of the unit, then (n = 16) the scaling; n = 32
+// adds the cross-lane stage h = 16 (every lane of the warp must take part)
+// before it.  `odd` = this unit is the upper half of its 32-value block.
+template <int N>
+__device__ __forceinline__ void rotate_unit(float f[16], float scale, bool odd) {
+  unsigned long long P[8];
+  fwht16_packed(f, P);
   if (N == 32) {
     // lower half: own + other; upper half: other - own (= own * -1 + other)
     const float sg = odd ? -1.0f : 1.0f;
@@ -212,6 +217,21 @@ __device__ __forceinline__ void rotate_unit(float f[16], float scale, bool odd) 
   const unsigned long long SC = f2(scale, scale);   // a power of two: exact
 #pragma unroll
   for (int k = 0; k < 8; ++k) f2_split(mul_f2(P[k], SC), f[2 * k], f[2 * k + 1]);
+}
+
+// A whole 32-value block in one thread, held as two 16-value halves: the
+// stages of both halves, then h = 16 (lo + hi, lo - hi) and the scaling, all
+// as packed pairs; the same roundings as rotate_unit<32> on a lane pair.
+__device__ __forceinline__ void rotate_block32(float lo[16], float hi[16], float scale) {
+  unsigned long long A[8], B[8];
+  fwht16_packed(lo, A);
+  fwht16_packed(hi, B);
+  const unsigned long long SC = f2(scale, scale);   // a power of two: exact
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    f2_split(mul_f2(add_f2(A[k], B[k]), SC), lo[2 * k], lo[2 * k + 1]);
+    f2_split(mul_f2(sub_f2(A[k], B[k]), SC), hi[2 * k], hi[2 * k + 1]);
+  }
 }
 
 // Largest magnitude of 16 floats as binary32 magnitude bits (Inf and NaN

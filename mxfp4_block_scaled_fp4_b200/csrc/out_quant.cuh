@@ -64,18 +64,6 @@ __device__ __forceinline__ float col_scale(float a, const float* sigma_w, int n,
   return __fmul_rn(a, n < N ? __ldg(sigma_w + n) : 0.0f);
 }
 
-// In-thread rotation of a 32-value block held as two 16-value halves.
-__device__ __forceinline__ void rotate32_in_thread(float lo[16], float hi[16], float scale) {
-  rotate_unit<16>(lo, 1.0f, false);
-  rotate_unit<16>(hi, 1.0f, false);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float a = lo[i], b = hi[i];
-    lo[i] = __fmul_rn(__fadd_rn(a, b), scale);   // scale: a power of two, exact
-    hi[i] = __fmul_rn(__fsub_rn(a, b), scale);
-  }
-}
-
 // One row's BN output columns [n0, n0 + BN) as packed bf16 (word i = columns
 // 2i, 2i+1): quantize and store them.  row_real: row < M (codes and scales);
 // a row of the last 128-row block past M (MMA order) gets zero scales.
@@ -122,7 +110,7 @@ __device__ __forceinline__ void quant_out_row(const QuantOut& q, const QuantOutG
         unpack16(make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]), lo);
         unpack16(make_uint4(w[8], w[9], w[10], w[11]), make_uint4(w[12], w[13], w[14], w[15]), hi);
         if (q.rot == 32) {
-          rotate32_in_thread(lo, hi, q.rot_scale);
+          rotate_block32(lo, hi, q.rot_scale);
         } else {
           rotate_unit<16>(lo, q.rot_scale, false);
           rotate_unit<16>(hi, q.rot_scale, false);

@@ -332,6 +332,80 @@ __device__ __forceinline__ void quantize_units(const QuantArgs& a, long long u_b
   }
 }
 
+// The 32-rotation's quantize pass with a whole 32-value block per lane
+// (units 2b, 2b + 1 of block b): the rotation runs in the thread
+// (rotate_block32, no lane exchange), then the block's scale(s) and codes.
+// Blocks [u_begin / 2, u_end / 2) in slabs of 2 x 32 blocks per warp step
+// (128 units, as quantize_units), 4 loads per lane and block.
+template <int FMT, int LAYOUT>
+__device__ __forceinline__ void quantize_blocks32(const QuantArgs& a, long long u_begin,
+                                                  long long u_end, long long w, long long nwarps,
+                                                  bool reverse, int upr, FastDiv upr_div, int nsf,
+                                                  int ncb, float six_g, float y6, bool fast_b,
+                                                  const float* r_tab) {
+  const bool big = u_end > 0xFFFFFFFFll;
+  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
+  uint4* __restrict__ codes = reinterpret_cast<uint4*>(a.codes);
+  uint8_t* __restrict__ scales = a.scales;
+  const int lane = threadIdx.x & 31;
+  const long long b_begin = u_begin >> 1, b_end = u_end >> 1;
+  const long long n_slabs = (b_end - b_begin + 63) / 64;
+  for (long long t = w; t < n_slabs; t += nwarps) {
+    const long long slab = reverse ? n_slabs - 1 - t : t;
+    uint4 xs[2][4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const long long b = b_begin + slab * 64 + j * 32 + lane;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        xs[j][k] = (b < b_end) ? ld_stream(x + b * 32 + 8 * k) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const long long b = b_begin + slab * 64 + j * 32 + lane;
+      float lo[16], hi[16];
+      unpack16(xs[j][0], xs[j][1], lo);
+      unpack16(xs[j][2], xs[j][3], hi);
+      rotate_block32(lo, hi, a.rot_scale);
+      const unsigned m0 = mag_max16(lo), m1 = mag_max16(hi);
+      unsigned s0, s1 = 0u;
+      uint4 packed;
+      if (FMT == 0) {
+        s0 = nvfp4_scale_byte_f32(m0, six_g, y6, fast_b);
+        s1 = nvfp4_scale_byte_f32(m1, six_g, y6, fast_b);
+        const float r0 = r_tab[s0 & 127u], r1 = r_tab[s1 & 127u];
+        packed.x = r0 == 0.0f ? 0u : quant8_f32(lo, r0);
+        packed.y = r0 == 0.0f ? 0u : quant8_f32(lo + 8, r0);
+        packed.z = r1 == 0.0f ? 0u : quant8_f32(hi, r1);
+        packed.w = r1 == 0.0f ? 0u : quant8_f32(hi + 8, r1);
+      } else {
+        float r;
+        s0 = mxfp4_scale_f32(max(m0, m1), a.rule, &r);
+        packed = make_uint4(quant8_f32(lo, r), quant8_f32(lo + 8, r), quant8_f32(hi, r),
+                            quant8_f32(hi + 8, r));
+      }
+      if (b < b_end) {
+        codes[b] = packed;   // units 2b, 2b + 1
+        const long long u = 2 * b;
+        const long long row =
+            big ? u / upr : static_cast<long long>(fast_div(static_cast<unsigned>(u), upr_div));
+        const int jj = static_cast<int>(u - row * upr);   // even: a block never spans rows
+        if (FMT == 0) {
+          // scale columns jj, jj + 1: adjacent bytes, an aligned 16-bit word
+          // (in the MMA order jj % 4 is 0 or 2; row-major rows hold an even
+          // number of scales)
+          const long long off = (LAYOUT == 1) ? row * nsf + jj : mma_scale_offset(row, jj, ncb);
+          *reinterpret_cast<uint16_t*>(scales + off) = static_cast<uint16_t>(s0 | (s1 << 8));
+        } else {
+          const int c = jj >> 1;
+          const long long off = (LAYOUT == 1) ? row * nsf + c : mma_scale_offset(row, c, ncb);
+          scales[off] = static_cast<uint8_t>(s0);
+        }
+      }
+    }
+  }
+}
+
 // MMA order: zero the padding, columns [nsf, 4 ncb) of real rows, then every
 // column of rows [rows, rows padded to 128); items i = first, first + stride...
 __device__ __forceinline__ void zero_mma_padding(const QuantArgs& a, long long pad_a,
@@ -379,8 +453,12 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long
   }
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long gwarp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  quantize_units<FMT, LAYOUT, ROT>(a, 0, units, gwarp, stride >> 5, a.dynamic != 0, upr, upr_div,
+  if (ROT == 32)
+    quantize_blocks32<FMT, LAYOUT>(a, 0, units, gwarp, stride >> 5, a.dynamic != 0, upr, upr_div,
                                    nsf, ncb, six_g, y6, fast_b, r_tab);
+  else
+    quantize_units<FMT, LAYOUT, ROT>(a, 0, units, gwarp, stride >> 5, a.dynamic != 0, upr,
+                                     upr_div, nsf, ncb, six_g, y6, fast_b, r_tab);
   if (LAYOUT == 0)
     zero_mma_padding(a, pad_a, pad_b, nsf, ncb,
                      static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x, stride);
