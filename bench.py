@@ -527,6 +527,12 @@ def measure_prefill_matrix(torch, L, ops, a_big, w_big, dev, fp4_peak):
 MOE_CONFIGS = [(8, 16384, 4096, 4096), (64, 16384, 2048, 4096)]
 
 
+def cool_down(torch, dev, seconds=2.0):
+    """Lets the GPU idle for a moment between supplementary measurements."""
+    torch.cuda.synchronize(dev)
+    time.sleep(seconds)
+
+
 def grouped_kernel_name(M, N, E, sms=148):
     """The kernel fp4_gemm_grouped launches for M routed rows over E groups
     (its launch rule: the CTA-pair form when groups average 512 rows or more
@@ -579,10 +585,14 @@ def measure_grouped(torch, ops, dev, fp4_peak):
                     ops.gemm(sq, one, out=c[lo:hi])
 
             res = {}
+            clk = None
             for name, fn in (("grouped", grouped), ("separate_calls", separate)):
                 for _ in range(3):
                     fn()
                 ts = []
+                if name == "grouped":
+                    clk = Clocks(dev.index or 0)
+                    clk.start()
                 for _ in range(20):
                     flush_l2(torch, flush, flush_r)
                     e0 = torch.cuda.Event(enable_timing=True)
@@ -592,8 +602,12 @@ def measure_grouped(torch, ops, dev, fp4_peak):
                     e1.record()
                     torch.cuda.synchronize(dev)
                     ts.append(e0.elapsed_time(e1))
+                if name == "grouped":
+                    clk = clk.stop()
                 res[name] = float(np.median(ts))
             rows.append({"E": E, "M_routed": M, "N": N, "K": Kx,
+                         "sm_mhz_during_grouped": clk.get("sm_mhz"),
+                         "throttle_reasons": clk.get("reasons"),
                          "format": "NVFP4" if fmt == 0 else "MXFP4",
                          "group_rows_min_max": [int(sizes.min()), int(sizes.max())],
                          "grouped_ms": round(res["grouped"], 4),
@@ -1077,9 +1091,15 @@ def main():
                 "h2d_bytes_per_step": a_host.numel() * 2, "d2h_bytes_per_step": c_host.numel() * 2},
     }
     if not args.no_suite and (M, N, K) == (8192, 28672, 8192):
+        # each supplementary part starts after a short idle, so that the
+        # 1 kW power cap that the previous part's seconds of dense GEMMs
+        # engage has released (the grouped rows record their clocks)
         line["prefill_matrix"] = measure_prefill_matrix(torch, L, ops, a, w_dev, dev, fp4_peak)
+        cool_down(torch, dev)
         line["gemm_quant"] = measure_gemm_quant(torch, ops, a, w_dev, dev, fp4_peak)
+        cool_down(torch, dev)
         line["grouped"] = measure_grouped(torch, ops, dev, fp4_peak)
+        cool_down(torch, dev)
         line["mbs"] = measure_mbs(torch, ops, a, w_dev, dev, fp4_peak)
     if not args.no_suite:
         line["decode"] = measure_decode(torch, ops, L, inputs, dev, peaks["hbm_gbs"])

@@ -147,7 +147,8 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const uint4* __restri
 
 // The amax pass over rotated values: warps take slabs of 4 x 32 units of 16
 // values (every lane issues its 8 loads first), rotate each unit and keep
-// the largest magnitude (binary32 bits).
+// the largest magnitude (binary32 bits).  The 32-rotation gives each lane a
+// whole 32-value block instead (2 x 32 blocks per slab, rotate_block32).
 template <int ROT>
 __global__ void __launch_bounds__(kThreads, 4) amax_rot_kernel(const uint4* __restrict__ x,
                                                                long long n_units, float scale,
@@ -160,23 +161,42 @@ __global__ void __launch_bounds__(kThreads, 4) amax_rot_kernel(const uint4* __re
   const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   unsigned m = 0;
   for (long long t = gwarp; t < n_slabs; t += nwarps) {
-    uint4 v[4][2];
+    if (ROT == 32) {
+      const long long n_blocks = n_units >> 1;
+      uint4 v[2][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const long long u = t * 128 + j * 32 + lane;
-      if (u < n_units) {
-        v[j][0] = ld_stream(x + 2 * u);
-        v[j][1] = ld_stream(x + 2 * u + 1);
-      } else {
-        v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < 2; ++j) {
+        const long long b = t * 64 + j * 32 + lane;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[j][k] = (b < n_blocks) ? ld_stream(x + 4 * b + k) : make_uint4(0, 0, 0, 0);
       }
-    }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float f[16];
-      unpack16(v[j][0], v[j][1], f);
-      rotate_unit<ROT>(f, scale, (lane & 1) != 0);
-      m = max(m, mag_max16(f));
+      for (int j = 0; j < 2; ++j) {
+        float lo[16], hi[16];
+        unpack16(v[j][0], v[j][1], lo);
+        unpack16(v[j][2], v[j][3], hi);
+        rotate_block32(lo, hi, scale);
+        m = max(m, max(mag_max16(lo), mag_max16(hi)));
+      }
+    } else {
+      uint4 v[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const long long u = t * 128 + j * 32 + lane;
+        if (u < n_units) {
+          v[j][0] = ld_stream(x + 2 * u);
+          v[j][1] = ld_stream(x + 2 * u + 1);
+        } else {
+          v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float f[16];
+        unpack16(v[j][0], v[j][1], f);
+        rotate_unit<ROT>(f, scale, (lane & 1) != 0);
+        m = max(m, mag_max16(f));
+      }
     }
   }
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
