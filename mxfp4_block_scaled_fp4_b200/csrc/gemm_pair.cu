@@ -79,7 +79,7 @@ constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = 256;
 constexpr uint32_t SF_STAGE_COLS = 48;
 constexpr int kThreads = 352;       // 11 warps
-constexpr int GROUP_M = 16;             // raster: 16 tile rows (4096 rows of A) share W in L2
+constexpr int GROUP_M = 32;             // raster: 32 tile rows (8192 rows of A) share W in L2
 
 static_assert(SF_COL + STAGES * SF_STAGE_COLS <= TMEM_COLS, "scale stages exceed tensor memory");
 static_assert(SMEM_BYTES <= 227 * 1024, "ring exceeds shared memory");
