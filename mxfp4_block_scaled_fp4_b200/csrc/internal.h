@@ -62,6 +62,9 @@ struct QuantArgs {
   // DYNAMIC, small tensors: every quantize CTA takes the magnitude maximum
   // of the whole tensor itself (no amax pass, no partial maxima)
   int self_amax = 0;
+  // x is 32-byte aligned: a lane's 32 contiguous bytes come in one load
+  // (set by launch_quantize)
+  int wide = 0;
   // The status word a non-finite DYNAMIC maximum is reported in (set by
   // launch_quantize when null).
   unsigned* status = nullptr;

@@ -34,6 +34,26 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return v;
 }
 
+// 32 contiguous bytes of a lane: one 256-bit load when `wide` (the tensor is
+// 32-byte aligned), else two 16-byte loads.  A warp's 16-byte loads at a
+// lane stride above 16 bytes each touch part of every sector, and the next
+// load refetches them from L2 (no L1 allocation); the 256-bit load reads a
+// lane's sectors once.  Measured on B200 it pays where a lane reads 64
+// contiguous bytes (the 32-rotation's blocks: 8192 x 16384 MXFP4 + Hadamard-32
+// 67.6 -> 63.5 us) and not at 32 (the 16-value units: 2-6% slower), so only
+// the block pass uses it.
+__device__ __forceinline__ void ld_stream32(const void* p, bool wide, uint4& a, uint4& b) {
+  if (wide) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z),
+                   "=r"(b.w)
+                 : "l"(p));
+  } else {
+    a = ld_stream(p);
+    b = ld_stream(static_cast<const uint4*>(p) + 1);
+  }
+}
+
 // Byte offset of scale (row r, column c) in the MMA-consumable order.
 __device__ __forceinline__ long long mma_scale_offset(long long r, int c, int ncb) {
   const long long atom = (r >> 7) * ncb + (c >> 2);
@@ -376,9 +396,12 @@ __device__ __forceinline__ void quantize_blocks32(const QuantArgs& a, long long 
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const long long b = b_begin + slab * 64 + j * 32 + lane;
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        xs[j][k] = (b < b_end) ? ld_stream(x + b * 32 + 8 * k) : make_uint4(0, 0, 0, 0);
+      if (b < b_end) {
+        ld_stream32(x + b * 32, a.wide != 0, xs[j][0], xs[j][1]);
+        ld_stream32(x + b * 32 + 16, a.wide != 0, xs[j][2], xs[j][3]);
+      } else {
+        xs[j][0] = xs[j][1] = xs[j][2] = xs[j][3] = make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -576,6 +599,8 @@ QuantGeom quant_geom(const QuantArgs& a) {
 cudaError_t launch_quantize(const QuantArgs& a_in, cudaStream_t s, bool pdl) {
   QuantArgs a = a_in;
   if (!a.status && !(a.status = watchdog_ptr())) return cudaErrorInvalidSymbol;
+  // rows are 64-byte multiples (K % 32 == 0): the base decides the alignment
+  a.wide = (reinterpret_cast<uintptr_t>(a.x) % 32) == 0 ? 1 : 0;
   const QuantGeom q = quant_geom(a);
   const long long want = std::max((q.units + kThreads * 4 - 1) / (kThreads * 4),
                                   (q.pad_a + q.pad_b + kThreads - 1) / kThreads);
