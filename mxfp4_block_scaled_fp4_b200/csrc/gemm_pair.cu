@@ -138,7 +138,8 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mt, int
 // (out_quant.cuh), with the bf16 C stored as well when p.C is not null;
 // 4 / 5 = bf16 / fp32 C scaled by sigma_a[m] sigma_w[n] (MXFP4 macro-block
 // scaling) instead of alpha.
-template <int FMT, int OUT, int G = 0>
+// QROT (OUT 2, 3): the emitted activation's rotation order (0, 16, 32).
+template <int FMT, int OUT, int G = 0, int QROT = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_w,
@@ -644,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) bulk_wait_read_0();   // every earlier store has read its buffer
           __syncwarp();
           const uint32_t srow = row0 < p.M ? smem_u32(qbuf) + lane * 128 : 0u;
-          quant_out_row<BN, QOUT ? OUT - 2 : 0>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N,
+          quant_out_row<BN, QOUT ? OUT - 2 : 0, QROT>(p.qo, qg, packed, row, row_ok, pad, nt * BN, p.N,
                                                 srow, lane & 7);
           if (row0 < p.M) {
             fence_proxy_async_smem();
@@ -720,11 +721,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------ host side
 
-template <int FMT, int OUT, int G = 0>
+template <int FMT, int OUT, int G = 0, int QROT = 0>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc,
                          const CUtensorMap& mq,
                          const Params& p, int tiles, int max_sms, cudaStream_t s) {
-  auto kern = gemm_pair_kernel<FMT, OUT, G>;
+  auto kern = gemm_pair_kernel<FMT, OUT, G, QROT>;
   constexpr int SMEM_BYTES = PairLayout<G>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -845,9 +846,18 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s) {
   const int tiles = p.m_tiles * p.n_tiles;
   using L = cudaError_t (*)(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                             const CUtensorMap&, const Params&, int, int, cudaStream_t);
-  static const L table[2][4] = {
-      {launch_typed<0, 0>, launch_typed<0, 1>, launch_typed<0, 2>, launch_typed<0, 3>},
-      {launch_typed<1, 0>, launch_typed<1, 1>, launch_typed<1, 2>, launch_typed<1, 3>}};
+  static const L table[2][2] = {{launch_typed<0, 0>, launch_typed<0, 1>},
+                                {launch_typed<1, 0>, launch_typed<1, 1>}};
+  // the FP4-emitting epilogue, by operand format, output format and rotation
+  static const L qtable[2][2][3] = {
+      {{launch_typed<0, 2, 0, 0>, launch_typed<0, 2, 0, 16>, launch_typed<0, 2, 0, 32>},
+       {launch_typed<0, 3, 0, 0>, launch_typed<0, 3, 0, 16>, launch_typed<0, 3, 0, 32>}},
+      {{launch_typed<1, 2, 0, 0>, launch_typed<1, 2, 0, 16>, launch_typed<1, 2, 0, 32>},
+       {launch_typed<1, 3, 0, 0>, launch_typed<1, 3, 0, 16>, launch_typed<1, 3, 0, 32>}}};
+  if (a.out_mode == 2 || a.out_mode == 3) {
+    const int ri = a.qo.rot == 32 ? 2 : (a.qo.rot == 16 ? 1 : 0);
+    return qtable[a.fmt != 0][a.out_mode - 2][ri](ma, mw, mc, mq, p, tiles, a.max_sms, s);
+  }
   if (a.out_mode >= 4) {   // macro-block scaling: MXFP4 only
     if (a.fmt != 1) return cudaErrorInvalidValue;
     return a.out_mode == 5 ? launch_typed<1, 5>(ma, mw, mc, ma, p, tiles, a.max_sms, s)

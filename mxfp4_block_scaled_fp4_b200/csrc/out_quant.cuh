@@ -71,8 +71,11 @@ __device__ __forceinline__ float col_scale(float a, const float* sigma_w, int n,
 // written as zero by the tile that covers them.  N % 32 == 0.
 // srow != 0: the row's BN / 2 code bytes go to shared memory at srow (16-byte
 // chunk j at srow + ((j ^ swz) << 4), the 128-byte swizzle of a TMA store
-// box) instead of global memory; the caller stores the box.
-template <int BN, int FMT>
+// box) instead of global memory; the caller stores the box.  ROT: the
+// rotation order fixed at compile time (0: none, 16, 32), or -1 for q.rot at
+// run time (a kernel that instantiates one rotation keeps no registers for
+// the others).
+template <int BN, int FMT, int ROT = -1>
 __device__ __forceinline__ void quant_out_row(const QuantOut& q, const QuantOutG& gc,
                                               const uint32_t* packed, long long row, bool row_real,
                                               bool row_pad, int n0, int N, uint32_t srow = 0u,
@@ -88,7 +91,8 @@ __device__ __forceinline__ void quant_out_row(const QuantOut& q, const QuantOutG
     unsigned s0 = 0u, s1 = 0u;
     if (row_real && col < N) {
       const uint32_t* w = packed + 8 * u;
-      if (q.rot == 0) {
+      const int rot = ROT >= 0 ? ROT : q.rot;
+      if (rot == 0) {
         unsigned m0 = fold_u16x2(max_u16x2(mag_max8(make_uint4(w[0], w[1], w[2], w[3])),
                                            mag_max8(make_uint4(w[4], w[5], w[6], w[7]))));
         unsigned m1 = fold_u16x2(max_u16x2(mag_max8(make_uint4(w[8], w[9], w[10], w[11])),
@@ -109,7 +113,7 @@ __device__ __forceinline__ void quant_out_row(const QuantOut& q, const QuantOutG
         float lo[16], hi[16];
         unpack16(make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]), lo);
         unpack16(make_uint4(w[8], w[9], w[10], w[11]), make_uint4(w[12], w[13], w[14], w[15]), hi);
-        if (q.rot == 32) {
+        if (rot == 32) {
           rotate_block32(lo, hi, q.rot_scale);
         } else {
           rotate_unit<16>(lo, q.rot_scale, false);
