@@ -519,19 +519,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // accumulator is released before any global store is issued
           uint32_t packed[BN / 2];
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            uint32_t r[32];
-            FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
+          for (int c = 0; c < BN / 16; ++c) {
+            uint32_t r[16];
+            FP4_TMEM_LD_32x32b_X16(tbase + c * 16, r);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int n = nt * BN + 32 * c + 2 * j;
+            for (int j = 0; j < 8; ++j) {
+              const int n = nt * BN + 16 * c + 2 * j;
               const float lo =
                   __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n, p.N), __uint_as_float(r[2 * j]));
               const float hi =
                   __fmul_rn(col_scale<MBS>(arow, p.sigma_w, n + 1, p.N), __uint_as_float(r[2 * j + 1]));
               __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-              packed[16 * c + j] = *reinterpret_cast<uint32_t*>(&h);
+              packed[8 * c + j] = *reinterpret_cast<uint32_t*>(&h);
             }
           }
           tc_fence_before();

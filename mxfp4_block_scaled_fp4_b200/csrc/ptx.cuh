@@ -405,6 +405,16 @@ __host__ __device__ constexpr uint32_t idesc_fp4(uint32_t M, uint32_t N, bool e8
          (e8m0_scales ? 1u : 0u) << 23 | ((M >> 4) & 0x1Fu) << 24 | (a_sf_id & 3u) << 29;
 }
 
+// 32 lanes x 16 consecutive fp32 columns of tensor memory -> registers.
+#define FP4_TMEM_LD_32x32b_X16(taddr, r)                                                   \
+  asm volatile(                                                                            \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "                                            \
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"                     \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),            \
+        "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),          \
+        "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])                                 \
+      : "r"(taddr))
+
 // 32 lanes x 32 consecutive fp32 columns of tensor memory -> registers.
 #define FP4_TMEM_LD_32x32b_X32(taddr, r)                                                   \
   asm volatile(                                                                            \
