@@ -519,15 +519,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!F32) {
           uint32_t packed[BN / 2];
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            uint32_t r[32];
-            FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
+          for (int c = 0; c < BN / 16; ++c) {
+            uint32_t r[16];
+            FP4_TMEM_LD_32x32b_X16(tbase + c * 16, r);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 8; ++j) {
               __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r[2 * j])),
                                                        __fmul_rn(alpha, __uint_as_float(r[2 * j + 1])));
-              packed[16 * c + j] = *reinterpret_cast<uint32_t*>(&h);
+              packed[8 * c + j] = *reinterpret_cast<uint32_t*>(&h);
             }
           }
           tc_fence_before();
@@ -585,18 +585,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!F32) {
         uint32_t packed[BN / 2];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          FP4_TMEM_LD_32x32b_X32(tbase + c * 32, r);
+        for (int c = 0; c < BN / 16; ++c) {
+          uint32_t r[16];
+          FP4_TMEM_LD_32x32b_X16(tbase + c * 16, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int jc = 32 * c + 2 * j;   // column within the tile
+          for (int j = 0; j < 8; ++j) {
+            const int jc = 16 * c + 2 * j;   // column within the tile
             const float lo = __fmul_rn(MBS ? __fmul_rn(arow, sw[jc]) : arow, __uint_as_float(r[2 * j]));
             const float hi =
                 __fmul_rn(MBS ? __fmul_rn(arow, sw[jc + 1]) : arow, __uint_as_float(r[2 * j + 1]));
             __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-            packed[16 * c + j] = *reinterpret_cast<uint32_t*>(&h);
+            packed[8 * c + j] = *reinterpret_cast<uint32_t*>(&h);
           }
         }
         tc_fence_before();
