@@ -56,7 +56,7 @@ FP4_NOMINAL_TFLOPS = 9000.0   # B200 dense FP4 tensor peak, nominal (context)
 # takes (gemm_pair_kernel), measured with ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass).  None whenever that kernel has changed
 # since it was last measured.
-GEMM_TRAFFIC_BYTES = 274.9e6 + 442.6e6
+GEMM_TRAFFIC_BYTES = 264.9e6 + 441.7e6
 
 
 def gemm_kernel_name(m, n, k):
