@@ -360,8 +360,9 @@ fp4_status_t fp4_quantize_act_noalloc(const void* x, int rows, int K, fp4_format
  * out (bits 0-6) and when a DYNAMIC global-scale reduction meets a
  * non-finite input (bit 7, FP4_STATUS_NONFINITE_BIT).  A bit set by a kernel
  * on another stream is never lost: it is either returned by this call or
- * left for the next.  Synchronizes `stream` (the exchange runs on it after
- * the work queued before).  *code receives the raw word (0 = nothing
+ * left for the next, also when several host threads call this at once
+ * (their calls are serialized).  Synchronizes `stream` (the exchange runs on
+ * it after the work queued before).  *code receives the raw word (0 = nothing
  * happened).  Returns FP4_ERR_DEVICE_TIMEOUT if a wait ran out, else
  * FP4_ERR_NONFINITE if only the non-finite bit was set, else FP4_OK.
  * Non-finite inputs are outside the format's contract ("Hardware FP4

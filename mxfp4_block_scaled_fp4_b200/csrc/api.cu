@@ -3,7 +3,9 @@
 // quantize.cu, gemm.cu and fused.cu.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
+#include <mutex>
 
 #include "fp4.h"
 #include "internal.h"
@@ -15,8 +17,11 @@ namespace fp4 {
 // (the WD_* codes of ptx.cuh) or when a DYNAMIC amax meets a non-finite
 // input (WD_NONFINITE).
 static __device__ unsigned int g_watchdog = 0;
-// Where fp4_device_status's exchange leaves the word it took.
+// Where fp4_device_status's exchange leaves the word it took.  One slot for
+// all callers: g_status_mutex keeps a second call's exchange from
+// overwriting it before the first call has copied it out.
 static __device__ unsigned int g_status_taken = 0;
+static std::mutex g_status_mutex;
 
 // Takes the status word and clears it in one atomic exchange, so that a bit
 // a kernel on another stream sets meanwhile is never lost.
@@ -24,16 +29,20 @@ __global__ void status_take_kernel(unsigned* wd, unsigned* taken) {
   *taken = atomicExch(wd, 0u);
 }
 
+// The word's address on the current device (looked up once per device;
+// concurrent first calls store the same address).
 unsigned* watchdog_ptr() {
-  static unsigned* cached[64] = {nullptr};
+  static std::atomic<unsigned*> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cached[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_watchdog) != cudaSuccess) return nullptr;
-    cached[dev] = static_cast<unsigned*>(p);
+  unsigned* p = cached[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_watchdog) != cudaSuccess) return nullptr;
+    p = static_cast<unsigned*>(q);
+    cached[dev].store(p, std::memory_order_release);
   }
-  return cached[dev];
+  return p;
 }
 
 // The watchdog self-test: one warp waits on an mbarrier that nothing
@@ -68,16 +77,18 @@ fp4_status_t check_rows_k(long long rows, int K) {
 }
 
 fp4_status_t device_ok() {
-  static int cached[64] = {0};   // 0 unknown, 1 ok, 2 bad
+  static std::atomic<int> cached[64] = {};   // 0 unknown, 1 ok, 2 bad
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP4_ERR_NO_DEVICE;
-  if (cached[dev] == 0) {
+  int c = cached[dev].load(std::memory_order_relaxed);
+  if (c == 0) {
     int major = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
       return FP4_ERR_NO_DEVICE;
-    cached[dev] = (major == 10) ? 1 : 2;
+    c = (major == 10) ? 1 : 2;
+    cached[dev].store(c, std::memory_order_relaxed);
   }
-  return cached[dev] == 1 ? FP4_OK : FP4_ERR_NO_DEVICE;
+  return c == 1 ? FP4_OK : FP4_ERR_NO_DEVICE;
 }
 
 size_t quant_ws_bytes() { return fp4::quant_workspace_bytes(); }
@@ -484,6 +495,7 @@ fp4_status_t fp4_device_status(unsigned* code, void* stream) {
   if ((st = device_ok()) != FP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned* wd = fp4::watchdog_ptr();
+  std::lock_guard<std::mutex> lock(fp4::g_status_mutex);
   void* taken = nullptr;
   if (!wd || cudaGetSymbolAddress(&taken, fp4::g_status_taken) != cudaSuccess) return FP4_ERR_CUDA;
   fp4::status_take_kernel<<<1, 1, 0, s>>>(wd, static_cast<unsigned*>(taken));

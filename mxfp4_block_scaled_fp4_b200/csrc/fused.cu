@@ -412,16 +412,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 // Packed codes [rows, K/2] as a 2-D uint8 tensor, boxes of 128 bytes x
 // box_rows rows, 128-byte swizzle; out-of-range rows and columns read as 0.
 bool make_map(CUtensorMap* m, const uint8_t* base, int rows, int K, int box_rows) {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  // the driver's encoder, looked up once (thread-safe static initialization)
+  static const EncodeTiledFn fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
             cudaSuccess ||
         q != cudaDriverEntryPointSuccess)
-      return false;
-    fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
+  if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(FBK_BYTES), static_cast<cuuint32_t>(box_rows)};

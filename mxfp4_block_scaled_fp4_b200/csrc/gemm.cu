@@ -37,6 +37,7 @@
 // word, the CTA stops issuing, waits (bounded) for its copies and MMAs in
 // flight, frees its tensor memory and returns.
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cuda_bf16.h>
 
@@ -686,16 +687,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once (a function-local static
+// is initialized once even when threads race to the first call).
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  static const EncodeTiledFn fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
   return fn;
 }
 
@@ -777,10 +780,11 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const Par
 // once (cached per device, width and size; 0 when the query fails).
 template <int BN>
 int max_clusters(int size) {
-  static int cache[64][9] = {};
+  static std::atomic<int> cache[64][9] = {};
   int dev = 0;
   if (size < 2 || size > 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (cache[dev][size] == 0) {
+  int c = cache[dev][size].load(std::memory_order_relaxed);
+  if (c == 0) {
     auto kern = gemm_kernel<0, 0, BN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<BN>::SMEM) !=
         cudaSuccess)
@@ -801,9 +805,10 @@ int max_clusters(int size) {
       (void)cudaGetLastError();
       return 0;
     }
-    cache[dev][size] = n > 0 ? n : -1;
+    c = n > 0 ? n : -1;
+    cache[dev][size].store(c, std::memory_order_relaxed);
   }
-  return cache[dev][size] > 0 ? cache[dev][size] : 0;
+  return c > 0 ? c : 0;
 }
 
 int max_clusters_bn(int bn, int size) {

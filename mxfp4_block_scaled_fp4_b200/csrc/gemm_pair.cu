@@ -45,6 +45,7 @@
 // both CTAs, the leader waits for its MMAs in flight, and both CTAs meet at
 // a final cluster barrier before the pair's tensor memory is freed.
 #include <algorithm>
+#include <atomic>
 #include <cuda_bf16.h>
 
 #include "groups.cuh"
@@ -741,20 +742,20 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mw, const CUt
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // pairs that fit on the device at once (cached per device and form)
-  static int max_pairs[64] = {0};
+  static std::atomic<int> max_pairs[64] = {};
   int dev = 0;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (max_pairs[dev] <= 0) {
+  int fit = max_pairs[dev].load(std::memory_order_relaxed);
+  if (fit <= 0) {
     cfg.gridDim = dim3(2);
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&fit, kern, &cfg);
     if (e != cudaSuccess) return e;
-    if (n <= 0) return cudaErrorInvalidConfiguration;
-    max_pairs[dev] = n;
+    if (fit <= 0) return cudaErrorInvalidConfiguration;
+    max_pairs[dev].store(fit, std::memory_order_relaxed);
   }
-  const int pairs = std::max(1, std::min({tiles, max_pairs[dev], gemm_sms(max_sms) / 2}));
+  const int pairs = std::max(1, std::min({tiles, fit, gemm_sms(max_sms) / 2}));
   cfg.gridDim = dim3(2 * pairs);
   e = cudaLaunchKernelEx(&cfg, kern, ma, mw, mc, mq, p);
   if (e != cudaSuccess) return e;

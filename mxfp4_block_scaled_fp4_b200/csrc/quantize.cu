@@ -16,6 +16,7 @@
 // warp are contiguous.  All floating-point steps use explicitly rounded
 // intrinsics (no contraction), one IEEE binary32 rounding per step.
 #include <algorithm>
+#include <atomic>
 
 #include "internal.h"
 #include "codec.cuh"
@@ -510,16 +511,16 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a, long
 }  // namespace
 
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 namespace {
