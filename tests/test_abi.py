@@ -1,6 +1,7 @@
 """The C ABI without a GPU: the library loads, exports every function the
-header declares, and its host-only functions (sizes, argument checks, status
-strings) behave as documented.  No compute call is made here."""
+header declares, the ctypes binding matches the header's prototypes, and the
+host-only functions (sizes, argument checks, status strings) behave as
+documented.  No compute call is made here."""
 import ctypes
 
 import pytest
@@ -120,3 +121,48 @@ def test_quant_options_checked_before_any_launch(lib):
     fx = L.fp4_gemm_fused_ex
     assert fx(fake, fake, fake, fake, 8, 16, 256, 0, 0, L.opts(64, 0), fake, fake, 16, 0, fake,
               1 << 30, 0, None) == L.FP4_ERR_INVALID_ARG
+
+
+def _header_prototypes():
+    import re
+    with open(L.HEADER) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    out = {}
+    for ret, name, params in re.findall(
+            r"([A-Za-z_][A-Za-z0-9_ \*]*?)\b(fp4_[a-z_]+)\s*\(([^)]*)\)\s*;", text):
+        ps = [p.strip() for p in params.split(",")] if params.strip() not in ("", "void") else []
+        out[name] = (ret.strip(), ps)
+    return out
+
+
+def _kind_of_c(t):
+    """pointer / 64-bit unsigned (size_t, unsigned long long) / 32-bit int
+    or enum, from a C parameter or return declaration."""
+    if "*" in t:
+        return "ptr"
+    if "unsigned long long" in t or "size_t" in t:
+        return "u64"
+    return "int"
+
+
+def _kind_of_ctypes(t):
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or isinstance(getattr(t, "_type_", None), type):
+        return "ptr"
+    if t in (ctypes.c_ulonglong, ctypes.c_size_t) and ctypes.sizeof(t) == 8:
+        return "u64"
+    assert t is ctypes.c_int, t
+    return "int"
+
+
+def test_binding_matches_header_prototypes():
+    """Every binding's argument list has the header's parameter count and,
+    parameter by parameter, the same kind (pointer, size_t, 64-bit, int or
+    enum); so do the return types."""
+    protos = _header_prototypes()
+    assert set(protos) == set(L.SIGNATURES)
+    for name, (ret, params) in protos.items():
+        res, args = L.SIGNATURES[name]
+        assert len(args) == len(params), (name, len(args), len(params))
+        for i, (c, py) in enumerate(zip(params, args)):
+            assert _kind_of_c(c) == _kind_of_ctypes(py), (name, i, c, py)
+        assert _kind_of_c(ret) == _kind_of_ctypes(res), (name, ret, res)
