@@ -41,6 +41,19 @@ def _check(status: int, what: str):
         raise L.Fp4Error(status, what)
 
 
+def _check_out(out: torch.Tensor, M: int, N: int, device: torch.device):
+    """A caller's output must be exactly [M, N] (rows may be strided: the
+    leading dimension is out.stride(0)), unit-stride along N, bf16 or fp32,
+    on the operands' device -- the kernels write M x N values through it."""
+    if out.dim() != 2 or tuple(out.shape) != (M, N) or (N > 1 and out.stride(1) != 1):
+        raise ValueError(f"out must be [{M}, {N}] with unit stride along N, got "
+                         f"{tuple(out.shape)} strides {tuple(out.stride())}")
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bf16 or fp32")
+    if out.device != device:
+        raise ValueError(f"out is on {out.device}, the operands on {device}")
+
+
 def _cuda_bf16_2d(t: torch.Tensor, name: str):
     if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous 2-D bf16 CUDA tensor")
@@ -137,6 +150,7 @@ def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
     dev = a.codes.device
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    _check_out(out, M, N, dev)
     o = L.FP4_OUT_F32 if out.dtype == torch.float32 else L.FP4_OUT_BF16
     if a.sigma is not None:
         _check(L.fp4_gemm_mbs(a.codes.data_ptr(), a.scales.data_ptr(), a.sigma.data_ptr(),
@@ -217,11 +231,13 @@ def gemm_grouped(a: Quantized, w: QuantizedExperts, offsets: torch.Tensor,
     activation times expert e's weights.  offsets: int32 CUDA tensor [E+1]."""
     if a.fmt != w.fmt or a.K != w.K or a.layout != SCALES_MMA:
         raise ValueError("operands must share format and K and use the MMA scale layout")
-    if (not offsets.is_cuda or offsets.dtype != torch.int32 or offsets.numel() != w.E + 1):
-        raise ValueError("offsets must be an int32 CUDA tensor of E + 1 entries")
+    if (not offsets.is_cuda or offsets.dtype != torch.int32 or offsets.numel() != w.E + 1
+            or not offsets.is_contiguous()):
+        raise ValueError("offsets must be a contiguous int32 CUDA tensor of E + 1 entries")
     M, N, K = a.rows, w.N, a.K
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=a.codes.device)
+    _check_out(out, M, N, a.codes.device)
     o = L.FP4_OUT_F32 if out.dtype == torch.float32 else L.FP4_OUT_BF16
     _check(L.fp4_gemm_grouped(a.codes.data_ptr(), a.scales.data_ptr(), a.g.data_ptr(),
                               w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(),
@@ -252,6 +268,7 @@ def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
     dev = x.device
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    _check_out(out, M, N, dev)
     o = L.FP4_OUT_F32 if out.dtype == torch.float32 else L.FP4_OUT_BF16
     gmode = L.FP4_GLOBAL_DYNAMIC if g_a is None else L.FP4_GLOBAL_STATIC
     if g_a is None:
