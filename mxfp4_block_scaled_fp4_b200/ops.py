@@ -54,6 +54,31 @@ def _check_out(out: torch.Tensor, M: int, N: int, device: torch.device):
         raise ValueError(f"out is on {out.device}, the operands on {device}")
 
 
+def _check_scalar(t: torch.Tensor, name: str, device: torch.device):
+    """A global scale the kernels read (or write) at t.data_ptr()."""
+    if t.dtype != torch.float32 or t.numel() < 1 or t.device != device:
+        raise ValueError(f"{name} must be a float32 tensor of at least one element on {device}")
+
+
+def _check_quantized(q: "Quantized", name: str, device: torch.device):
+    """The buffers of a quantized operand must hold what the kernels read:
+    codes uint8 [rows, K/2], at least fp4_scale_bytes scale bytes, a float32
+    global scale (and rows macro-block scales), all on one device."""
+    if (q.codes.dtype != torch.uint8 or tuple(q.codes.shape) != (q.rows, q.K // 2)
+            or not q.codes.is_contiguous()):
+        raise ValueError(f"{name}.codes must be contiguous uint8 [{q.rows}, {q.K // 2}]")
+    need = L.fp4_scale_bytes(q.rows, q.K, q.fmt, q.layout)
+    if q.scales.dtype != torch.uint8 or not q.scales.is_contiguous() or q.scales.numel() < need:
+        raise ValueError(f"{name}.scales must be contiguous uint8 of at least {need} bytes")
+    _check_scalar(q.g, f"{name}.g", device)
+    if q.sigma is not None and (q.sigma.dtype != torch.float32 or q.sigma.numel() < q.rows
+                                or not q.sigma.is_contiguous()):
+        raise ValueError(f"{name}.sigma must be contiguous float32 of at least {q.rows} values")
+    for t in (q.codes, q.scales) + ((q.sigma,) if q.sigma is not None else ()):
+        if t.device != device:
+            raise ValueError(f"{name} has buffers on {t.device}, expected {device}")
+
+
 def _cuda_bf16_2d(t: torch.Tensor, name: str):
     if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous 2-D bf16 CUDA tensor")
@@ -89,6 +114,7 @@ def quantize(x: torch.Tensor, fmt: int = NVFP4, layout: int = SCALES_MMA,
                          device=dev)
     gmode = L.FP4_GLOBAL_DYNAMIC if g is None else L.FP4_GLOBAL_STATIC
     gt = torch.ones(1, dtype=torch.float32, device=dev) if g is None else g
+    _check_scalar(gt, "g", dev)
     ws_bytes = L.fp4_workspace_bytes(rows, 0, K, fmt)
     if ws is None:
         ws = workspace(ws_bytes, dev)
@@ -148,6 +174,8 @@ def gemm(a: Quantized, w: Quantized, out_dtype=torch.bfloat16,
         raise ValueError("macro-block scaling needs both operands quantized with it")
     M, N, K = a.rows, w.rows, a.K
     dev = a.codes.device
+    _check_quantized(a, "a", dev)
+    _check_quantized(w, "w", dev)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=dev)
     _check_out(out, M, N, dev)
@@ -177,11 +205,14 @@ def gemm_quant(a: Quantized, w: Quantized, out_fmt: int = NVFP4, out_layout: int
         raise ValueError("a rotated activation needs weights rotated with the same order")
     M, N, K = a.rows, w.rows, a.K
     dev = a.codes.device
+    _check_quantized(a, "a", dev)
+    _check_quantized(w, "w", dev)
     codes = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty(max(L.fp4_scale_bytes(M, N, out_fmt, out_layout), 1), dtype=torch.uint8,
                          device=dev)
     if g_out is None:
         g_out = torch.ones(1, dtype=torch.float32, device=dev)
+    _check_scalar(g_out, "g_out", dev)
     c = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if with_c else None
     _check(L.fp4_gemm_quant(a.codes.data_ptr(), a.scales.data_ptr(), a.g.data_ptr(),
                             w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(), M, N, K,
@@ -235,9 +266,21 @@ def gemm_grouped(a: Quantized, w: QuantizedExperts, offsets: torch.Tensor,
             or not offsets.is_contiguous()):
         raise ValueError("offsets must be a contiguous int32 CUDA tensor of E + 1 entries")
     M, N, K = a.rows, w.N, a.K
+    dev = a.codes.device
+    _check_quantized(a, "a", dev)
+    sfb = L.fp4_scale_bytes(N, K, w.fmt, SCALES_MMA)
+    if (w.codes.dtype != torch.uint8 or tuple(w.codes.shape) != (w.E, N, K // 2)
+            or not w.codes.is_contiguous() or w.scales.dtype != torch.uint8
+            or tuple(w.scales.shape) != (w.E, sfb) or not w.scales.is_contiguous()
+            or w.g.dtype != torch.float32 or w.g.numel() < w.E
+            or any(t.device != dev for t in (w.codes, w.scales, w.g))):
+        raise ValueError(f"experts must be uint8 codes [{w.E}, {N}, {K // 2}], uint8 scales "
+                         f"[{w.E}, {sfb}] and float32 g [{w.E}], contiguous, on {dev}")
+    if offsets.device != dev:
+        raise ValueError(f"offsets are on {offsets.device}, the operands on {dev}")
     if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=a.codes.device)
-    _check_out(out, M, N, a.codes.device)
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    _check_out(out, M, N, dev)
     o = L.FP4_OUT_F32 if out.dtype == torch.float32 else L.FP4_OUT_BF16
     _check(L.fp4_gemm_grouped(a.codes.data_ptr(), a.scales.data_ptr(), a.g.data_ptr(),
                               w.codes.data_ptr(), w.scales.data_ptr(), w.g.data_ptr(),
@@ -266,6 +309,9 @@ def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
     M, K = x.shape
     N = w.rows
     dev = x.device
+    _check_quantized(w, "w", dev)
+    if K != w.K:
+        raise ValueError(f"x has K = {K}, w has K = {w.K}")
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=dev)
     _check_out(out, M, N, dev)
@@ -273,6 +319,7 @@ def gemm_fused(x: torch.Tensor, w: Quantized, out_dtype=torch.bfloat16,
     gmode = L.FP4_GLOBAL_DYNAMIC if g_a is None else L.FP4_GLOBAL_STATIC
     if g_a is None:
         g_a = g_out if g_out is not None else torch.ones(1, dtype=torch.float32, device=dev)
+    _check_scalar(g_a, "g_a" if gmode == L.FP4_GLOBAL_STATIC else "g_out", dev)
     need = L.fp4_workspace_bytes(M, N, K, w.fmt)
     if ws is None:
         ws = workspace(need, dev)
