@@ -540,7 +540,7 @@ def grouped_kernel_name(M, N, E, sms=148):
     pair_ctas = 2 * (-(-M // 256)) * (-(-N // 256))
     if M >= 512 * E and N > 128 and M > 128 and 2 * pair_ctas >= sms:
         return "fp4 gemm_pair_kernel grouped (256x256 tiles on CTA pairs"
-    return ("fp4 gemm_kernel grouped (128x256 tiles" if E <= 128 and N > 128 else
+    return ("fp4 gemm_kernel grouped (128x256 tiles" if N > 128 else
             "fp4 gemm_kernel grouped (128x128 tiles")
 
 

@@ -305,8 +305,9 @@ fp4_status_t fp4_gemm_mbs(const uint8_t* a_codes, const uint8_t* a_scales, const
  *               outside A and C is read or written.
  * 1 <= E <= 256, N % 8 == 0, K % 32 == 0.  Empty groups are allowed.  Every
  * tile has all of K (no split): 256 x 256 tiles on CTA pairs when the
- * groups average at least 512 rows (M >= 512 E), else 128 x 256 tiles
- * (E <= 128, N > 128) or 128 x 128.  ws unused (may be NULL).
+ * groups average at least 512 rows (M >= 512 E), N > 128 and the pair
+ * tiles keep at least half the SMs busy, else 128 x 256 tiles (N > 128) or
+ * 128 x 128.  ws unused (may be NULL).
  * "FP4 n'existe pas : il existe des FP4, et chaque runtime choisit son
  * dialecte", section "Les runtimes et leurs dialectes : qui parle quoi"
  * (fused NVFP4 MoE kernels, W4A4 MegaMoE). */

@@ -65,5 +65,6 @@ def test_grouped_kernel_name_follows_the_launch_rule():
     # smaller groups: 128-row tiles, 256 wide unless N <= 128
     assert "128x256" in bench.grouped_kernel_name(16384, 2048, 64)
     assert "128x128" in bench.grouped_kernel_name(16384, 128, 8)
+    assert "128x256" in bench.grouped_kernel_name(16384, 384, 256)   # any E up to 256
     # too few pair tiles for half the SMs: 128-row tiles
     assert "gemm_kernel" in bench.grouped_kernel_name(1024, 256, 1)
